@@ -1,0 +1,188 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 linear-layer library.
+ *
+ * NVFP4 as this library stores it (aisight.pl, "Koniec marnowania mocy.
+ * NVIDIA udowadnia, ze 4 bity wystarcza do trenowania gigantow", section
+ * "Architektura NVFP4 kontra ograniczenia mikroskalowania": blocks of 16
+ * elements instead of 32, an E4M3 block scale instead of a power of two, and
+ * an extra FP32 scale for the whole tensor):
+ *   - codes : E2M1 values (+-{0,0.5,1,1.5,2,3,4,6}), two per byte, element 2i
+ *             in bits 0-3 and element 2i+1 in bits 4-7, row-major
+ *             [rows x k/2] bytes ("K-major": k, the GEMM reduction index, is
+ *             contiguous);
+ *   - scales: one unsigned E4M3 byte per 16 consecutive k of a row, stored in
+ *             512-byte atoms of 128 rows x 4 blocks: byte offset of (row r,
+ *             block b) = atom * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + b % 4
+ *             with atom = (r / 128) * (KB / 4) + b / 4, KB = 4 * ceil(k / 64).
+ *             Rows are padded to 128 and blocks to KB; padding bytes are 0.
+ *             This is the order in which the tensor cores read block scales;
+ *   - tensor_scale: one FP32 decode scale s_t in device memory.
+ * A value decodes as e2m1(code) * e4m3(scale) * s_t.
+ *
+ * Conventions for every call:
+ *   - Pointers to tensors are DEVICE pointers on the current CUDA device; the
+ *     caller allocates and owns every buffer (inputs, outputs, workspace).
+ *     The library allocates nothing and frees nothing.
+ *   - Calls are asynchronous and stream-ordered on `stream` (0 = legacy
+ *     default stream); none synchronises the host.
+ *   - Arguments are checked on the host before anything is launched; a call
+ *     that returns an error has launched nothing and written nothing.
+ *   - A workspace serves one stream at a time.  Its first 256 bytes hold a
+ *     device status word: zero it once after allocation.  Kernels with bounded
+ *     device-side waits record NVFP4_ERR_DEVICE_TIMEOUT there instead of
+ *     hanging; nvfp4_check() reads and clears it.
+ *   - Non-finite inputs are outside the contract (the result is unspecified).
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVFP4_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+typedef enum nvfp4_status {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum/flag combination */
+    NVFP4_ERR_ALIGNMENT = 2,          /* pointer or leading dimension breaks the 16-byte rule   */
+    NVFP4_ERR_SHAPE = 3,              /* sizes the format or the kernels cannot take            */
+    NVFP4_ERR_WORKSPACE = 4,          /* workspace missing or smaller than required             */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 5, /* current device is not compute capability 10.0          */
+    NVFP4_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed                   */
+    NVFP4_ERR_DEVICE_TIMEOUT = 7      /* a bounded device-side wait expired (see nvfp4_check)   */
+} nvfp4_status;
+
+typedef enum nvfp4_dtype {
+    NVFP4_DTYPE_F32 = 0,  /* IEEE binary32 */
+    NVFP4_DTYPE_BF16 = 1  /* bfloat16      */
+} nvfp4_dtype;
+
+enum { NVFP4_ROWWISE = 0, NVFP4_COLWISE = 1 };
+enum { NVFP4_RTN = 0, NVFP4_SR = 1 };
+
+/* An NVFP4 tensor of logical shape [rows x k] (k = reduction dim). */
+typedef struct nvfp4_tensor {
+    uint8_t *codes;       /* nvfp4_codes_bytes(rows, k) bytes, 16-byte aligned  */
+    uint8_t *scales;      /* nvfp4_scales_bytes(rows, k) bytes, 16-byte aligned */
+    float *tensor_scale;  /* 1 float                                            */
+    int64_t rows;
+    int64_t k;
+} nvfp4_tensor;
+
+/* Sizes of the two byte buffers of an NVFP4 tensor (k must be a multiple of 16). */
+NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t k);
+NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t k);
+
+/* Workspace bytes needed by nvfp4_quantize (status word + per-CTA amax partials). */
+NVFP4_API size_t nvfp4_quantize_workspace_size(void);
+
+/*
+ * nvfp4_quantize -- x [R x C] (row-major, leading dimension ld elements) -> out.
+ * The step order follows aisight.pl, sections "Architektura NVFP4 ..." and
+ * "Technologie stabilizujace proces treningowy":
+ *   1. optional 16-point random Hadamard transform y = 1/4 H16 D v of every
+ *      16-element block (D = +-1 signs from the seed), colwise only;
+ *   2. tensor amax over the (transformed) tensor, unless amax_in supplies it;
+ *      s_t = amax / (6 * 448) (1 if that is 0);
+ *   3. per 16-block: sb = E4M3_rn_satfinite(amax_b / 6 / s_t);
+ *   4. per element: r = v * (1 / (e4m3(sb) * s_t)), then E2M1 by
+ *      round-to-nearest-even (rounding = NVFP4_RTN) or stochastic rounding
+ *      (NVFP4_SR: up iff u < frac, u a 16-bit Philox4x32-10 draw keyed on
+ *      (seed, element index in the output view));
+ *   5. store codes, scales (atom layout, padding zeroed) and s_t.
+ * orientation = NVFP4_ROWWISE: blocks run along the C columns; out is
+ *   [R x C] (out->rows == R, out->k == C).  Requires C % 16 == 0.
+ * orientation = NVFP4_COLWISE: blocks run down the R rows and out is the
+ *   transpose [C x R] (out->rows == C, out->k == R).  Requires R % 16 == 0
+ *   and C a multiple of 8 (bf16) / 4 (f32).
+ * rht != 0 only with NVFP4_COLWISE.  x must be 16-byte aligned and
+ * ld * element size a multiple of 16.  workspace: >= nvfp4_quantize_workspace_size()
+ * bytes (may be NULL when amax_in is given).  amax_in: optional device float.
+ * R == 0 or C == 0 is allowed: only s_t = 1 is written.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
+                            int orientation, int rounding, int rht, uint64_t seed,
+                            const float *amax_in, const nvfp4_tensor *out,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * nvfp4_gemm -- C[M x N] = (A . B^T) * sA * sB with A = [M x K], B = [N x K]
+ * NVFP4 tensors (the block-scaled GEMM used for Fprop, Dgrad and Wgrad; 4-bit
+ * GEMMs on Blackwell tensor cores: nerdman.de, "Nvidia drueckt KI-Training auf
+ * 4 Bit runter", section "Was konkret passiert ist").  Products of E2M1 values
+ * and E4M3 block scales accumulate in FP32 on the tensor cores; the epilogue
+ * multiplies by the two tensor scales and writes c_dtype (f32 or bf16,
+ * round-to-nearest-even) row-major with leading dimension ldc elements.
+ * Requires A->k == B->k, K % 64 == 0, C 16-byte aligned, ldc * element size a
+ * multiple of 16.  M or N == 0: nothing is done.  K == 0: C is zero-filled.
+ * workspace: >= 256 bytes (status word).
+ */
+NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
+                        int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes for nvfp4_linear_fwd / nvfp4_linear_bwd at these sizes. */
+NVFP4_API size_t nvfp4_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvfp4_linear_fwd -- Fprop of Y = X . W^T: X [M x K], W [N x K] (dtype,
+ * row-major, contiguous) -> Y [M x N] (y_dtype, contiguous).  Both operands
+ * are quantised rowwise with round-to-nearest-even, then nvfp4_gemm.
+ * Requires K % 64 == 0; quantised operands live in the workspace.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
+                              nvfp4_dtype dtype, nvfp4_dtype y_dtype,
+                              void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * nvfp4_linear_bwd -- backward of Y = X . W^T, with dY [M x N], X [M x K],
+ * W [N x K] (dtype, contiguous):
+ *   Dgrad dX [M x K] (dx_dtype) = dY . W :  A = rowwise(dY, RTN), B = colwise(W, RTN)
+ *   Wgrad dW [N x K] (f32)      = dY^T . X: A = colwise(dY, RHT, SR), B = colwise(X, RHT, RTN)
+ * The random Hadamard transform and stochastic rounding apply to the Wgrad
+ * operands only (aisight.pl, section "Technologie stabilizujace proces
+ * treningowy"); both Wgrad operands use the same signs, from `seed`, which
+ * also keys the SR draws.  Requires M % 64 == 0, N % 64 == 0, K % 64 == 0.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void *dX, float *dW,
+                              int64_t M, int64_t N, int64_t K, nvfp4_dtype dtype,
+                              nvfp4_dtype dx_dtype, uint64_t seed,
+                              void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Squared-ReLU activation of the MLP block and its derivative, bf16 in/out,
+ * n elements, contiguous, 16-byte aligned:
+ *   h  = relu(y) * relu(y)          (binary32, then bf16 round-to-nearest-even)
+ *   dy = dh * (2 * relu(y))         (binary32, then bf16 round-to-nearest-even)
+ * with relu(y) = y for y > 0 and +0 otherwise.
+ */
+NVFP4_API nvfp4_status nvfp4_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t stream);
+NVFP4_API nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace's device status
+ * word: NVFP4_OK, NVFP4_ERR_DEVICE_TIMEOUT, or NVFP4_ERR_CUDA if the stream
+ * reports an error. */
+NVFP4_API nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream);
+
+/* Number of kernel launches the most recent successful call on this host
+ * thread issued (launch accounting for benchmarks). */
+NVFP4_API int nvfp4_last_launch_count(void);
+
+/* Static description of a status code. */
+NVFP4_API const char *nvfp4_status_string(nvfp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

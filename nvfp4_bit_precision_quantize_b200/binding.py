@@ -1,0 +1,224 @@
+"""Thin ctypes binding of libnvfp4.so (include/nvfp4.h).
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every computation runs in the library's CUDA kernels.  There is no
+CPU fallback: if the library is missing or the device is not a B200 the calls
+raise.  Function names follow the C ABI.
+"""
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
+
+NVFP4_OK = 0
+NVFP4_ERR_INVALID_ARG = 1
+NVFP4_ERR_ALIGNMENT = 2
+NVFP4_ERR_SHAPE = 3
+NVFP4_ERR_WORKSPACE = 4
+NVFP4_ERR_UNSUPPORTED_DEVICE = 5
+NVFP4_ERR_CUDA = 6
+NVFP4_ERR_DEVICE_TIMEOUT = 7
+
+NVFP4_DTYPE_F32 = 0
+NVFP4_DTYPE_BF16 = 1
+NVFP4_ROWWISE = 0
+NVFP4_COLWISE = 1
+NVFP4_RTN = 0
+NVFP4_SR = 1
+
+# Functions declared in include/nvfp4.h (checked by the tests against the header).
+EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_size", "nvfp4_quantize",
+           "nvfp4_gemm", "nvfp4_linear_workspace_size", "nvfp4_linear_fwd", "nvfp4_linear_bwd",
+           "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
+           "nvfp4_status_string")
+
+
+class CTensor(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("tensor_scale", C.c_void_p),
+                ("rows", C.c_int64), ("k", C.c_int64)]
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+_lib = None
+
+
+def load():
+    """Load libnvfp4.so (built in-tree by nvfp4_bit_precision_quantize_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libnvfp4.so is not built; run `python -m nvfp4_bit_precision_quantize_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    vp, i64, sz, i32, u64 = C.c_void_p, C.c_int64, C.c_size_t, C.c_int, C.c_uint64
+    tp = C.POINTER(CTensor)
+    sig = {
+        "nvfp4_codes_bytes": (sz, [i64, i64]),
+        "nvfp4_scales_bytes": (sz, [i64, i64]),
+        "nvfp4_quantize_workspace_size": (sz, []),
+        "nvfp4_quantize": (i32, [vp, i32, i64, i64, i64, i32, i32, i32, u64, vp, tp, vp, sz, vp]),
+        "nvfp4_gemm": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
+        "nvfp4_linear_workspace_size": (sz, [i64, i64, i64]),
+        "nvfp4_linear_fwd": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]),
+        "nvfp4_linear_bwd": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, u64, vp, sz, vp]),
+        "nvfp4_relu2_fwd": (i32, [vp, vp, i64, vp]),
+        "nvfp4_relu2_bwd": (i32, [vp, vp, vp, i64, vp]),
+        "nvfp4_check": (i32, [vp, vp]),
+        "nvfp4_last_launch_count": (i32, []),
+        "nvfp4_status_string": (C.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return _lib
+
+
+def status_string(status):
+    return load().nvfp4_status_string(int(status)).decode()
+
+
+def _ok(status, where):
+    if status != NVFP4_OK:
+        raise NVFP4Error(status, where)
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t == torch.bfloat16:
+        return NVFP4_DTYPE_BF16
+    if t == torch.float32:
+        return NVFP4_DTYPE_F32
+    raise TypeError("only float32 and bfloat16 are supported, got %s" % t)
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else None
+
+
+@dataclass
+class NVFP4Tensor:
+    """Device NVFP4 tensor [rows x k]: codes (uint8 [rows, k/2]), scales (uint8,
+    scale-atom layout), tensor_scale (float32 [1])."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tensor_scale: torch.Tensor
+    rows: int
+    k: int
+
+    def c(self):
+        return CTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.tensor_scale.data_ptr(),
+                       self.rows, self.k)
+
+
+def nvfp4_codes_bytes(rows, k):
+    return load().nvfp4_codes_bytes(rows, k)
+
+
+def nvfp4_scales_bytes(rows, k):
+    return load().nvfp4_scales_bytes(rows, k)
+
+
+def nvfp4_quantize_workspace_size():
+    return load().nvfp4_quantize_workspace_size()
+
+
+def nvfp4_linear_workspace_size(M, N, K):
+    return load().nvfp4_linear_workspace_size(M, N, K)
+
+
+def workspace(nbytes, device=None):
+    """A zeroed workspace (its status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def empty_nvfp4(rows, k, device=None):
+    device = device or "cuda"
+    return NVFP4Tensor(
+        codes=torch.empty((rows, k // 2), dtype=torch.uint8, device=device),
+        scales=torch.empty(max(nvfp4_scales_bytes(rows, k), 16), dtype=torch.uint8, device=device),
+        tensor_scale=torch.empty(1, dtype=torch.float32, device=device), rows=rows, k=k)
+
+
+def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, seed=1234, amax_in=None,
+                   out=None, ws=None, stream=None):
+    """Quantise a 2-D float32/bfloat16 CUDA tensor to NVFP4 (see include/nvfp4.h)."""
+    R, Cc = x.shape
+    rows, k = (Cc, R) if orientation == NVFP4_COLWISE else (R, Cc)
+    out = out or empty_nvfp4(rows, k, x.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), x.device)
+    ct = out.c()
+    st = load().nvfp4_quantize(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), orientation, rounding,
+                               int(bool(rht)), seed, _ptr(amax_in), C.byref(ct), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    _ok(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_gemm(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+    """C = (A . B^T) * sA * sB for NVFP4 tensors A [M x K], B [N x K]."""
+    M, N = A.rows, B.rows
+    out = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=A.codes.device)
+    ws = ws if ws is not None else workspace(256, A.codes.device)
+    ca, cb = A.c(), B.c()
+    st = load().nvfp4_gemm(C.byref(ca), C.byref(cb), _ptr(out), _dtype_code(out.dtype), out.stride(0), _ptr(ws),
+                           ws.numel(), _stream(stream))
+    _ok(st, "nvfp4_gemm")
+    return out
+
+
+def nvfp4_linear_fwd(X, W, y_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+    M, K = X.shape
+    N = W.shape[0]
+    out = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
+    ws = ws if ws is not None else workspace(nvfp4_linear_workspace_size(M, N, K), X.device)
+    st = load().nvfp4_linear_fwd(_ptr(X), _ptr(W), _ptr(out), M, N, K, _dtype_code(X.dtype),
+                                 _dtype_code(out.dtype), _ptr(ws), ws.numel(), _stream(stream))
+    _ok(st, "nvfp4_linear_fwd")
+    return out
+
+
+def nvfp4_linear_bwd(dY, X, W, seed=1234, dx_dtype=torch.bfloat16, dX=None, dW=None, ws=None, stream=None):
+    M, N = dY.shape
+    K = X.shape[1]
+    dX = dX if dX is not None else torch.empty((M, K), dtype=dx_dtype, device=X.device)
+    dW = dW if dW is not None else torch.empty((N, K), dtype=torch.float32, device=X.device)
+    ws = ws if ws is not None else workspace(nvfp4_linear_workspace_size(M, N, K), X.device)
+    st = load().nvfp4_linear_bwd(_ptr(dY), _ptr(X), _ptr(W), _ptr(dX), _ptr(dW), M, N, K, _dtype_code(X.dtype),
+                                 _dtype_code(dX.dtype), seed, _ptr(ws), ws.numel(), _stream(stream))
+    _ok(st, "nvfp4_linear_bwd")
+    return dX, dW
+
+
+def nvfp4_relu2_fwd(y, out=None, stream=None):
+    out = out if out is not None else torch.empty_like(y)
+    _ok(load().nvfp4_relu2_fwd(_ptr(y), _ptr(out), y.numel(), _stream(stream)), "nvfp4_relu2_fwd")
+    return out
+
+
+def nvfp4_relu2_bwd(dh, y, out=None, stream=None):
+    out = out if out is not None else torch.empty_like(y)
+    _ok(load().nvfp4_relu2_bwd(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _stream(stream)), "nvfp4_relu2_bwd")
+    return out
+
+
+def nvfp4_check(ws, stream=None):
+    """Synchronise and read/clear the workspace status word; raises on a device error."""
+    _ok(load().nvfp4_check(_ptr(ws), _stream(stream)), "nvfp4_check")
+
+
+def nvfp4_last_launch_count():
+    return load().nvfp4_last_launch_count()

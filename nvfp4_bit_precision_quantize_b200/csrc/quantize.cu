@@ -1,0 +1,404 @@
+// quantize.cu -- NVFP4 quantisation kernels for sm_100a.
+//
+// Two passes over the input, both HBM-bound:
+//   pass 1 (amax_*): tensor amax (after the random Hadamard transform when it
+//     is on), written as one partial per CTA -- no atomics, no zeroing;
+//   pass 2 (quantize_*): every CTA reduces the partials to the same amax,
+//     derives the FP32 tensor scale, and turns its tile into packed E2M1 codes
+//     plus E4M3 block scales laid out in the tensor cores' 128x4 scale atoms.
+// Format: aisight.pl, "Koniec marnowania mocy ...", section "Architektura
+// NVFP4 kontra ograniczenia mikroskalowania" (block 16, E4M3 block scale, FP32
+// tensor scale).  Hadamard transform and stochastic rounding on the Wgrad
+// operands: same page, section "Technologie stabilizujace proces treningowy".
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------------------
+// Pass 1a: max |x| over an [R x C] tensor (any orientation, no transform).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const T *__restrict__ x, int64_t R, int64_t C,
+                                                        int64_t ld, float *__restrict__ partials) {
+    constexpr int N = Vec<T>::N;
+    __shared__ float s_red[kThreads / 32];
+    const int64_t chunks_per_row = C / N;
+    const int64_t total = R * chunks_per_row;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    float m = 0.0f;
+    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (ld == C) {
+        constexpr int U = 4;  // independent 16-byte loads in flight per thread
+        for (; i + (U - 1) * stride < total; i += U * stride) {
+            uint4 raw[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) raw[u] = ldg_stream(x + (i + u * stride) * N);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float v[N];
+                Vec<T>::unpack(raw[u], v);
+#pragma unroll
+                for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+            }
+        }
+        for (; i < total; i += stride) {
+            float v[N];
+            Vec<T>::unpack(ldg_stream(x + i * N), v);
+#pragma unroll
+            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+        }
+    } else {
+        for (; i < total; i += stride) {
+            const int64_t r = i / chunks_per_row, c = (i - r * chunks_per_row) * N;
+            float v[N];
+            Vec<T>::unpack(ldg_stream(x + r * ld + c), v);
+#pragma unroll
+            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
+        partials[blockIdx.x] = b;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 1b: max |RHT(x)| where the transform runs down 16-row groups of every
+// column.  One work unit = one 16-row group x N columns (one 16-byte load per
+// row); consecutive threads take consecutive column chunks.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict__ x, int64_t R, int64_t C,
+                                                            int64_t ld, uint64_t seed,
+                                                            float *__restrict__ partials) {
+    constexpr int N = Vec<T>::N;
+    __shared__ float s_red[kThreads / 32];
+    const uint32_t signs = rht_sign_bits(seed);
+    const int64_t chunks = C / N;
+    const int64_t total = (R / 16) * chunks;
+    float m = 0.0f;
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * kThreads) {
+        const int64_t g = u / chunks, cc = u - g * chunks;
+        const T *p = x + (g * 16) * ld + cc * N;
+        uint4 raw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float t[N];
+                Vec<T>::unpack(raw[i], t);
+                v[i] = t[j];
+            }
+            rht16(v, signs);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
+        partials[blockIdx.x] = b;
+    }
+}
+
+struct QParams {
+    const void *x;
+    int64_t R, C, ld;
+    uint64_t seed;
+    const float *amax_in;
+    const float *partials;
+    int num_partials;
+    uint8_t *codes;
+    uint8_t *scales;
+    float *tensor_scale;
+};
+
+__device__ __forceinline__ float tensor_amax(const QParams &p, float *s_red) {
+    return p.amax_in ? *p.amax_in : reduce_partials_max(p.partials, p.num_partials, s_red);
+}
+
+// 16-bit SR draws for the 8 consecutive output-view indices idx0 .. idx0+7
+// (idx0 % 8 == 0): one Philox block keyed on the seed at counter (idx0 >> 3).
+__device__ __forceinline__ uint4 sr_words(uint64_t idx0, uint64_t seed) {
+    return philox4x32_10(make_uint4((uint32_t)(idx0 >> 3), (uint32_t)(idx0 >> 35), 0u, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+}
+__device__ __forceinline__ uint32_t rnd16_of(const uint4 &w, int e) {  // e = idx & 7
+    const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
+    return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2, rowwise: blocks of 16 along the contiguous columns.
+// CTA tile = 128 rows x (32*N) columns; warp w owns rows 16w..16w+15 and each
+// lane one 16-byte chunk of every row (2 (bf16) or 4 (f32) lanes per block).
+// Codes leave as one coalesced 128/64-byte segment per warp and row; the
+// tile's scale atoms are staged in shared memory and written as 16-byte pieces.
+// ---------------------------------------------------------------------------
+template <typename T, bool SR>
+__global__ void __launch_bounds__(kThreads) quantize_rowwise_kernel(const QParams p) {
+    constexpr int N = Vec<T>::N;
+    constexpr int LPB = 16 / N;          // lanes per 16-block
+    constexpr int TILE_C = 32 * N;
+    constexpr int ATOMS = TILE_C / 64;   // scale atoms per tile
+    __shared__ __align__(16) uint8_t s_sc[ATOMS * 512];
+    __shared__ float s_red[kThreads / 32];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rbase = (int64_t)blockIdx.y * 128 + warp * 16;
+    const int64_t c = (int64_t)blockIdx.x * TILE_C + lane * N;
+    const T *x = static_cast<const T *>(p.x);
+    const bool col_ok = c < p.C;
+
+    uint4 raw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int64_t r = rbase + i;
+        raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+    const int64_t K = p.C;
+    const int64_t KB4 = (K + 63) / 64;
+
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int64_t r = rbase + i;
+        float v[N];
+        Vec<T>::unpack(raw[i], v);
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        const BlockScale bs = block_scale(m, s_t);
+        float q[N];
+        if (SR) {
+            const uint64_t idx0 = (uint64_t)r * (uint64_t)K + (uint64_t)c;
+            const uint4 w = sr_words(idx0 & ~7ull, p.seed);
+            const int e0 = (int)(idx0 & 7);
+#pragma unroll
+            for (int j = 0; j < N; ++j)
+                q[j] = bs.zero ? 0.0f : sr_e2m1_value(__fmul_rn(v[j], bs.inv), rnd16_of(w, e0 + j));
+        } else {
+#pragma unroll
+            for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
+        }
+        if (col_ok && r < p.R) {
+            uint8_t *dst = p.codes + r * (K / 2) + c / 2;
+            if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
+            else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+        }
+        if ((lane % LPB) == 0) {
+            const int rl = warp * 16 + i, bl = lane / LPB;
+            s_sc[(bl >> 2) * 512 + (rl & 31) * 16 + ((rl >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)bs.sb;
+        }
+    }
+    __syncthreads();
+    const int64_t atom0 = (int64_t)blockIdx.x * ATOMS;
+    for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
+        const int atom = i >> 5;
+        if (atom0 + atom < KB4) {
+            uint8_t *dst = p.scales + ((int64_t)blockIdx.y * KB4 + atom0 + atom) * 512 + (i & 31) * 16;
+            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_sc + i * 16);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2, colwise: blocks of 16 run down the rows; the output is the transpose
+// ([C x R], K = R contiguous).  CTA tile = 256 rows x (32*N) columns; warp w
+// owns rows 32w..32w+31 (two 16-row groups) and each lane N adjacent columns,
+// so every block (one column x 16 rows) sits in one thread's registers: the
+// transform, block amax and encoding need no shuffles.  A lane's 16 code bytes
+// per column (two groups) form one 16-byte unit, staged in shared memory with
+// an xor swizzle so both the scatter and the row-contiguous read-out are free
+// of bank conflicts beyond the 4-wavefront minimum.
+// ---------------------------------------------------------------------------
+template <typename T, bool SR, bool RHT>
+__global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QParams p) {
+    constexpr int N = Vec<T>::N;
+    constexpr int W = kThreads / 32;     // warps
+    constexpr int TC = 32 * N;           // output rows per tile
+    constexpr int TR = 32 * W;           // k (input rows) per tile
+    constexpr int P = W;                 // 16-byte code units per output row per tile
+    constexpr int AR = TC / 128;         // scale-atom rows per tile
+    constexpr int AC = TR / 64;          // scale-atom columns per tile
+    __shared__ __align__(16) uint4 s_units[N * P * 32];
+    __shared__ __align__(16) uint8_t s_sc[AR * AC * 512];
+    __shared__ float s_red[W];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t c = (int64_t)blockIdx.x * TC + lane * N;
+    const int64_t r_warp = (int64_t)blockIdx.y * TR + warp * 32;
+    const T *x = static_cast<const T *>(p.x);
+    const bool col_ok = c < p.C;
+    const int64_t K = p.R;
+    const int64_t KB4 = (K + 63) / 64;
+
+    // issue the first group's loads before the amax reduction
+    uint4 raw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int64_t r = r_warp + i;
+        raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+    const uint32_t signs = RHT ? rht_sign_bits(p.seed) : 0u;
+
+    uint2 cw[N][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int64_t rg = r_warp + 16 * h;
+        if (h == 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int64_t r = rg + i;
+                raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float t[N];
+                Vec<T>::unpack(raw[i], t);
+                v[i] = t[j];
+            }
+            if (RHT) rht16(v, signs);
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+            const BlockScale bs = block_scale(m, s_t);
+            float q[16];
+            if (SR) {
+                const uint64_t idx0 = (uint64_t)(c + j) * (uint64_t)K + (uint64_t)rg;  // multiple of 16
+                const uint4 w0 = sr_words(idx0, p.seed), w1 = sr_words(idx0 + 8, p.seed);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    q[i] = bs.zero ? 0.0f
+                                   : sr_e2m1_value(__fmul_rn(v[i], bs.inv), rnd16_of(i < 8 ? w0 : w1, i & 7));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) q[i] = bs.zero ? 0.0f : __fmul_rn(v[i], bs.inv);
+            }
+            cw[j][h] = make_uint2(e2m1x8(q), e2m1x8(q + 8));
+            const int cl = lane * N + j, gl = warp * 2 + h;
+            s_sc[((cl >> 7) * AC + (gl >> 2)) * 512 + (cl & 31) * 16 + ((cl >> 5) & 3) * 4 + (gl & 3)] =
+                (uint8_t)bs.sb;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        const int q = j * P + warp;
+        s_units[q * 32 + (lane ^ (q & 7))] = make_uint4(cw[j][0].x, cw[j][0].y, cw[j][1].x, cw[j][1].y);
+    }
+    __syncthreads();
+
+    // codes: output row (c0 + cl) gets P units of 16 bytes at k-byte offset r0/2 + 16 p
+    const int64_t c0 = (int64_t)blockIdx.x * TC, r0 = (int64_t)blockIdx.y * TR;
+    const bool vec16 = (K % 32) == 0;
+    for (int i = threadIdx.x; i < TC * P; i += kThreads) {
+        const int cl = i / P, pu = i % P;
+        const int l = cl / N, j = cl % N, q = j * P + pu;
+        const int64_t orow = c0 + cl;
+        const int64_t rem = p.R - (r0 + 32 * pu);
+        if (orow < p.C && rem > 0) {
+            const uint4 u = s_units[q * 32 + (l ^ (q & 7))];
+            uint8_t *dst = p.codes + orow * (K / 2) + (r0 / 2) + 16 * pu;
+            if (rem >= 32 && vec16) {
+                *reinterpret_cast<uint4 *>(dst) = u;
+            } else {  // rows only 8-byte aligned (K % 32 == 16), or the K tail
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(u.x, u.y);
+                if (rem >= 32) *reinterpret_cast<uint2 *>(dst + 8) = make_uint2(u.z, u.w);
+            }
+        }
+    }
+    // scales: AR x AC atoms; each atom row's AC atoms are contiguous in memory
+    const int64_t rowtiles = (p.C + 127) / 128;
+    for (int i = threadIdx.x; i < AR * AC * 32; i += kThreads) {
+        const int atom = i >> 5, ar = atom / AC, ac = atom % AC;
+        const int64_t grow = (int64_t)blockIdx.x * AR + ar, gcol = (int64_t)blockIdx.y * AC + ac;
+        if (grow < rowtiles && gcol < KB4) {
+            uint8_t *dst = p.scales + (grow * KB4 + gcol) * 512 + (i & 31) * 16;
+            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_sc + i * 16);
+        }
+    }
+}
+
+// Empty tensor: only the tensor scale is defined.
+__global__ void tensor_scale_only_kernel(const float *amax_in, float *tensor_scale) {
+    *tensor_scale = tensor_scale_from_amax(amax_in ? *amax_in : 0.0f);
+}
+
+template <typename T>
+cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
+    const T *x = static_cast<const T *>(a.x);
+    int num_partials = 0;
+    if (!a.amax_in) {
+        const int sms = num_sms();
+        if (a.rht) {
+            const int64_t units = (a.R / 16) * (a.C / Vec<T>::N);
+            num_partials = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                                  std::max<int64_t>(1, (units + kThreads - 1) / kThreads));
+            amax_rht_kernel<T><<<num_partials, kThreads, 0, s>>>(x, a.R, a.C, a.ld, a.seed, a.partials);
+        } else {
+            const int64_t chunks = a.R * (a.C / Vec<T>::N);
+            num_partials = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                                  std::max<int64_t>(1, (chunks + kThreads - 1) / kThreads));
+            amax_kernel<T><<<num_partials, kThreads, 0, s>>>(x, a.R, a.C, a.ld, a.partials);
+        }
+        ++*launches;
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    QParams p{a.x, a.R, a.C, a.ld, a.seed, a.amax_in, a.partials, num_partials, a.codes, a.scales,
+              a.tensor_scale};
+    constexpr int N = Vec<T>::N;
+    if (!a.colwise) {
+        dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 127) / 128));
+        if (a.sr) quantize_rowwise_kernel<T, true><<<grid, kThreads, 0, s>>>(p);
+        else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);
+    } else {
+        dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 255) / 256));
+        if (a.sr && a.rht) quantize_colwise_kernel<T, true, true><<<grid, kThreads, 0, s>>>(p);
+        else if (a.sr) quantize_colwise_kernel<T, true, false><<<grid, kThreads, 0, s>>>(p);
+        else if (a.rht) quantize_colwise_kernel<T, false, true><<<grid, kThreads, 0, s>>>(p);
+        else quantize_colwise_kernel<T, false, false><<<grid, kThreads, 0, s>>>(p);
+    }
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches) {
+    if (a.R == 0 || a.C == 0) {
+        tensor_scale_only_kernel<<<1, 1, 0, s>>>(a.amax_in, a.tensor_scale);
+        ++*launches;
+        return cudaGetLastError();
+    }
+    return a.bf16 ? run<uint16_t>(a, s, launches) : run<float>(a, s, launches);
+}
+
+}  // namespace nvfp4

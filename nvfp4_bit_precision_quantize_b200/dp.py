@@ -1,0 +1,61 @@
+"""Data-parallel plumbing for the NVFP4 MLP step: one process per GPU.
+
+Each rank trains on its own token shard (weak scaling: the per-GPU batch is
+fixed) and the only exchange is the sum of the weight gradients dW across
+ranks (torch.distributed all-reduce; NCCL over NVLink on GPUs, gloo on CPU in
+the tests).  Timings are reduced as the maximum over ranks.
+"""
+import datetime
+import os
+
+import torch
+import torch.distributed as dist
+
+
+def world():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def init(backend="nccl", timeout_s=120):
+    """Join the process group if launched under torchrun (WORLD_SIZE > 1)."""
+    ws, rank, local = world()
+    if ws > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        kw = {}
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return ws, rank, local
+
+
+def shard_seed(base_seed, rank):
+    """Data seed of a rank's token shard (distinct shards, same weights)."""
+    return base_seed + 1000 * rank
+
+
+def allreduce_grads(grads):
+    """Sum each gradient tensor over all ranks, in place (no-op on one rank)."""
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        for g in grads:
+            dist.all_reduce(g, op=dist.ReduceOp.SUM)
+    return grads
+
+
+def max_over_ranks(value, device="cpu"):
+    """Maximum of a float over all ranks (the slowest rank sets the step time)."""
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return float(value)
+
+
+def barrier():
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def finish():
+    if dist.is_initialized():
+        dist.destroy_process_group()

@@ -55,6 +55,13 @@ def lib():
         L.oracle_bf16_from_f32.restype = C.c_uint16
         L.oracle_relu2_fwd.argtypes = [u16p, C.c_int64, u16p]
         L.oracle_relu2_bwd.argtypes = [u16p, u16p, C.c_int64, u16p]
+        L.oracle_amax.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_int,
+                                  C.c_int, C.c_uint64]
+        L.oracle_amax.restype = C.c_float
+        L.oracle_quantize_rows.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64,
+                                           C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_float,
+                                           i64p, C.c_int64, u8p, u8p]
+        L.oracle_quantize_rows.restype = C.c_int
         L.oracle_e2m1_rtn_array.argtypes = [f32p, C.c_int64, u8p]
         L.oracle_e2m1_sr_array.argtypes = [f32p, u32p, C.c_int64, u8p]
         L.oracle_e4m3_rn_array.argtypes = [f32p, C.c_int64, u8p]
@@ -173,6 +180,39 @@ def quantize(x, colwise=False, sr=False, rht=False, seed=1234, amax_in=None):
     if rc != 0:
         raise ValueError("oracle_quantize rejected the arguments")
     return codes, scales, ts[0], am[0]
+
+
+def _in(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return x, 1
+    if x.dtype == np.float32:
+        return x, 0
+    raise TypeError("x must be float32 or uint16 (bf16 bits)")
+
+
+def amax(x, colwise=False, rht=False, seed=1234):
+    """Tensor amax of the (optionally transformed) output view."""
+    x, bf16 = _in(x)
+    R, Cc = x.shape
+    return np.float32(lib().oracle_amax(x.ctypes.data_as(C.c_void_p), bf16, R, Cc, Cc, int(colwise),
+                                        int(rht), C.c_uint64(seed)))
+
+
+def quantize_rows(x, rows, amax_value, colwise=False, sr=False, rht=False, seed=1234):
+    """Codes and plain scales of selected output rows of the quantised tensor."""
+    x, bf16 = _in(x)
+    R, Cc = x.shape
+    K = R if colwise else Cc
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    codes = np.zeros((rows.size, K // 2), np.uint8)
+    scales = np.zeros((rows.size, K // 16), np.uint8)
+    rc = lib().oracle_quantize_rows(x.ctypes.data_as(C.c_void_p), bf16, R, Cc, Cc, int(colwise), int(sr),
+                                    int(rht), C.c_uint64(seed), float(amax_value), _p(rows, C.c_int64),
+                                    rows.size, _p(codes, C.c_uint8), _p(scales, C.c_uint8))
+    if rc != 0:
+        raise ValueError("oracle_quantize_rows rejected the arguments")
+    return codes, scales
 
 
 def dequantize(codes, scales, tensor_scale):

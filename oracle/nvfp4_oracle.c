@@ -276,6 +276,76 @@ unsigned oracle_block_scale(float amax_b, float s_t)
     return oracle_e4m3_rn_satfinite(t);
 }
 
+/* a1: tensor amax over the (optionally Hadamard-transformed) blocks of the
+ * output view.  Returns -1 on bad arguments. */
+float oracle_amax(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t ld,
+                  int colwise, int rht, uint64_t seed)
+{
+    int64_t rows = colwise ? C : R;
+    int64_t K = colwise ? R : C;
+    if (K % 16 != 0 || (rht && !colwise)) return -1.0f;
+    float d[16];
+    if (rht) oracle_rht_signs(seed, d);
+    float amax = 0.0f, v[16];
+    for (int64_t o = 0; o < rows; ++o)
+        for (int64_t b = 0; b < K / 16; ++b) {
+            load_block(x, dtype_bf16, ld, colwise, o, b, rht, d, v);
+            for (int j = 0; j < 16; ++j)
+                if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
+        }
+    return amax;
+}
+
+/* a2-a5 for one output row o, given the tensor scale s_t: writes the row's
+ * K/2 code bytes and K/16 scale bytes (plain order). */
+static void quantize_row(const void *x, int dtype_bf16, int64_t ld, int colwise, int sr, int rht,
+                         const float d[16], uint64_t seed, float s_t, int64_t o, int64_t K,
+                         uint8_t *codes_row, uint8_t *scales_row)
+{
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int64_t b = 0; b < K / 16; ++b) {
+        float v[16];
+        load_block(x, dtype_bf16, ld, colwise, o, b, rht, d, v);
+        /* a3: block amax and E4M3 block scale */
+        float amax_b = 0.0f;
+        for (int j = 0; j < 16; ++j)
+            if (fabsf(v[j]) > amax_b) amax_b = fabsf(v[j]);
+        unsigned sb = oracle_block_scale(amax_b, s_t);
+        scales_row[b] = (uint8_t)sb;
+        /* a4: element scale (reading: one reciprocal per block) */
+        float dec = (float)oracle_e4m3_value(sb) * s_t;
+        float inv = 1.0f / dec;
+        int zero_block = (sb == 0u) || (dec == 0.0f) || !isfinite(inv);
+        uint32_t words[4] = {0, 0, 0, 0};
+        int64_t have_group = -1;
+        for (int j = 0; j < 16; ++j) {
+            unsigned q = 0u;
+            if (!zero_block) {
+                float rr = v[j] * inv;
+                if (sr) {
+                    int64_t idx = o * K + b * 16 + j;   /* index in the output view */
+                    int64_t group = idx >> 3;
+                    if (group != have_group) {
+                        uint32_t ctr[4] = {(uint32_t)group, (uint32_t)(idx >> 35), 0u, 0u};
+                        oracle_philox4x32_10(ctr, key, words);
+                        have_group = group;
+                    }
+                    uint32_t w = words[(idx & 7) >> 1];
+                    uint32_t rnd16 = (idx & 1) ? (w >> 16) : (w & 0xFFFFu);
+                    q = oracle_e2m1_sr(rr, rnd16);
+                } else {
+                    q = oracle_e2m1_rtn(rr);
+                }
+            }
+            /* a5: pack, element 2i in the low nibble */
+            int64_t e = b * 16 + j;
+            uint8_t *byte = &codes_row[e >> 1];
+            if ((e & 1) == 0) *byte = (uint8_t)((*byte & 0xF0u) | q);
+            else              *byte = (uint8_t)((*byte & 0x0Fu) | (q << 4));
+        }
+    }
+}
+
 /* Quantise an [R x C] tensor (row-major, leading dimension ld, binary32 or
  * bf16 bits) to NVFP4.
  *   colwise = 0: output rows' = R, K = C, blocks along the columns.
@@ -296,71 +366,32 @@ int oracle_quantize(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t
     int64_t rows = colwise ? C : R;
     int64_t K = colwise ? R : C;
     if (K % 16 != 0 || rows < 0 || K < 0 || (rht && !colwise)) return -1;
-    int64_t nb = K / 16;
     float d[16];
     if (rht) oracle_rht_signs(seed, d);
-    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
-
-    /* a1: tensor amax over the (transformed) values */
-    float amax = 0.0f;
-    if (amax_in) {
-        amax = *amax_in;
-    } else {
-        float v[16];
-        for (int64_t o = 0; o < rows; ++o)
-            for (int64_t b = 0; b < nb; ++b) {
-                load_block(x, dtype_bf16, ld, colwise, o, b, rht, d, v);
-                for (int j = 0; j < 16; ++j)
-                    if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
-            }
-    }
+    float amax = amax_in ? *amax_in : oracle_amax(x, dtype_bf16, R, C, ld, colwise, rht, seed);
     float s_t = oracle_tensor_scale(amax);
     *tensor_scale = s_t;
     if (amax_out) *amax_out = amax;
+    for (int64_t o = 0; o < rows; ++o)
+        quantize_row(x, dtype_bf16, ld, colwise, sr, rht, d, seed, s_t, o, K,
+                     codes + o * (K / 2), scales + o * (K / 16));
+    return 0;
+}
 
-    for (int64_t o = 0; o < rows; ++o) {
-        for (int64_t b = 0; b < nb; ++b) {
-            float v[16];
-            load_block(x, dtype_bf16, ld, colwise, o, b, rht, d, v);
-            /* a3: block amax and E4M3 block scale */
-            float amax_b = 0.0f;
-            for (int j = 0; j < 16; ++j)
-                if (fabsf(v[j]) > amax_b) amax_b = fabsf(v[j]);
-            unsigned sb = oracle_block_scale(amax_b, s_t);
-            scales[o * nb + b] = (uint8_t)sb;
-            /* a4: element scale (reading: one reciprocal per block) */
-            float dec = (float)oracle_e4m3_value(sb) * s_t;
-            float inv = 1.0f / dec;
-            int zero_block = (sb == 0u) || (dec == 0.0f) || !isfinite(inv);
-            uint32_t words[4] = {0, 0, 0, 0};
-            int64_t have_group = -1;
-            for (int j = 0; j < 16; ++j) {
-                unsigned q = 0u;
-                if (!zero_block) {
-                    float rr = v[j] * inv;
-                    if (sr) {
-                        int64_t idx = o * K + b * 16 + j;
-                        int64_t group = idx >> 3;
-                        if (group != have_group) {
-                            uint32_t ctr[4] = {(uint32_t)group, (uint32_t)(idx >> 35), 0u, 0u};
-                            oracle_philox4x32_10(ctr, key, words);
-                            have_group = group;
-                        }
-                        uint32_t w = words[(idx & 7) >> 1];
-                        uint32_t rnd16 = (idx & 1) ? (w >> 16) : (w & 0xFFFFu);
-                        q = oracle_e2m1_sr(rr, rnd16);
-                    } else {
-                        q = oracle_e2m1_rtn(rr);
-                    }
-                }
-                /* a5: pack, element 2i in the low nibble */
-                int64_t e = o * K + b * 16 + j;
-                uint8_t *byte = &codes[e >> 1];
-                if ((e & 1) == 0) *byte = (uint8_t)((*byte & 0xF0u) | q);
-                else              *byte = (uint8_t)((*byte & 0x0Fu) | (q << 4));
-            }
-        }
-    }
+/* The same quantisation restricted to the output rows out_rows[i], i < n
+ * (for sampled checks of full-size tensors); amax is the tensor amax. */
+int oracle_quantize_rows(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t ld,
+                         int colwise, int sr, int rht, uint64_t seed, float amax,
+                         const int64_t *out_rows, int64_t n, uint8_t *codes, uint8_t *scales)
+{
+    int64_t K = colwise ? R : C;
+    if (K % 16 != 0 || (rht && !colwise)) return -1;
+    float d[16];
+    if (rht) oracle_rht_signs(seed, d);
+    float s_t = oracle_tensor_scale(amax);
+    for (int64_t i = 0; i < n; ++i)
+        quantize_row(x, dtype_bf16, ld, colwise, sr, rht, d, seed, s_t, out_rows[i], K,
+                     codes + i * (K / 2), scales + i * (K / 16));
     return 0;
 }
 

@@ -25,6 +25,7 @@ def cuda_lib():
     """The built C-ABI library, loaded through the binding (GPU tests only)."""
     if not _has_gpu():
         pytest.skip("no CUDA device")
-    from nvfp4_bit_precision_quantize_b200 import binding
+    from nvfp4_bit_precision_quantize_b200 import binding, build
+    build.build()
     binding.load()
     return binding

@@ -1,0 +1,115 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every
+function include/nvfp4.h declares, sizes match the documented layout, and
+invalid arguments are rejected before anything is launched."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from nvfp4_bit_precision_quantize_b200 import binding, build
+import layout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_sizes(lib):
+    assert lib.nvfp4_codes_bytes(256, 256) == 256 * 128
+    for rows, k in [(1, 16), (128, 64), (129, 64), (200, 272), (8192, 5120), (0, 64), (64, 0)]:
+        assert lib.nvfp4_scales_bytes(rows, k) == layout.scales_bytes(rows, k)
+    assert lib.nvfp4_quantize_workspace_size() >= 256 + 4 * 1024
+    assert lib.nvfp4_linear_workspace_size(8192, 20480, 5120) > 0.5625 * 8192 * 20480 * 2
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert len(binding.status_string(s)) > 0
+
+
+def _tensor(rows, k, codes=0x1000, scales=0x2000, ts=0x3000):
+    return binding.CTensor(codes, scales, ts, rows, k)
+
+
+def _q(lib, x=0x10000, dtype=1, R=64, Cc=64, ld=64, ori=0, rnd=0, rht=0, out=None, ws=0x20000,
+       wsb=1 << 20, amax=None):
+    out = out if out is not None else _tensor(R if ori == 0 else Cc, Cc if ori == 0 else R)
+    return lib.nvfp4_quantize(C.c_void_p(x), dtype, R, Cc, ld, ori, rnd, rht, 1234, amax, C.byref(out),
+                              C.c_void_p(ws), wsb, None)
+
+
+def test_quantize_rejections(lib):
+    E = binding
+    assert lib.nvfp4_quantize(C.c_void_p(0x10000), 1, 64, 64, 64, 0, 0, 0, 1, None, None, None, 0, None) \
+        == E.NVFP4_ERR_INVALID_ARG
+    assert _q(lib, x=0) == E.NVFP4_ERR_INVALID_ARG
+    assert _q(lib, dtype=7) == E.NVFP4_ERR_INVALID_ARG
+    assert _q(lib, ori=2) == E.NVFP4_ERR_INVALID_ARG
+    assert _q(lib, rnd=3) == E.NVFP4_ERR_INVALID_ARG
+    assert _q(lib, rht=1, ori=0) == E.NVFP4_ERR_INVALID_ARG          # RHT only colwise
+    assert _q(lib, Cc=40, ld=40) == E.NVFP4_ERR_SHAPE                # rowwise C % 16
+    assert _q(lib, R=40, ori=1, out=_tensor(64, 40)) == E.NVFP4_ERR_SHAPE  # colwise R % 16
+    assert _q(lib, ld=32) == E.NVFP4_ERR_SHAPE                       # ld < C
+    assert _q(lib, out=_tensor(64, 32)) == E.NVFP4_ERR_SHAPE         # output shape mismatch
+    assert _q(lib, R=-1) == E.NVFP4_ERR_SHAPE
+    assert _q(lib, x=0x10008) == E.NVFP4_ERR_ALIGNMENT
+    assert _q(lib, ld=72, Cc=64) == E.NVFP4_ERR_SHAPE or _q(lib, ld=68, Cc=64) == E.NVFP4_ERR_ALIGNMENT
+    assert _q(lib, ld=68, Cc=64) == E.NVFP4_ERR_ALIGNMENT            # 136-byte rows
+    assert _q(lib, out=_tensor(64, 64, codes=0x1004)) == E.NVFP4_ERR_ALIGNMENT
+    assert _q(lib, ws=0) == E.NVFP4_ERR_WORKSPACE
+    assert _q(lib, wsb=100) == E.NVFP4_ERR_WORKSPACE
+
+
+def test_gemm_rejections(lib):
+    E = binding
+    a, b = _tensor(128, 256), _tensor(256, 256)
+
+    def g(A=a, B=b, Cp=0x40000, dt=1, ldc=256, ws=0x50000, wsb=256):
+        return lib.nvfp4_gemm(C.byref(A), C.byref(B), C.c_void_p(Cp), dt, ldc, C.c_void_p(ws), wsb, None)
+    assert lib.nvfp4_gemm(None, C.byref(b), C.c_void_p(0x40000), 1, 256, C.c_void_p(0x50000), 256, None) \
+        == E.NVFP4_ERR_INVALID_ARG
+    assert g(B=_tensor(256, 128)) == E.NVFP4_ERR_SHAPE                # K mismatch
+    assert g(A=_tensor(128, 96), B=_tensor(256, 96)) == E.NVFP4_ERR_SHAPE  # K % 64
+    assert g(ldc=128) == E.NVFP4_ERR_SHAPE
+    assert g(Cp=0) == E.NVFP4_ERR_INVALID_ARG
+    assert g(Cp=0x40002) == E.NVFP4_ERR_ALIGNMENT
+    assert g(ldc=260) == E.NVFP4_ERR_ALIGNMENT                        # 520-byte bf16 rows
+    assert g(dt=5) == E.NVFP4_ERR_INVALID_ARG
+    assert g(ws=0) == E.NVFP4_ERR_WORKSPACE
+    assert g(A=_tensor(0, 256)) == E.NVFP4_OK                         # empty: nothing to do
+
+
+def test_linear_rejections(lib):
+    E = binding
+    ws = lib.nvfp4_linear_workspace_size(128, 128, 128)
+    p = C.c_void_p
+    assert lib.nvfp4_linear_fwd(p(0x1000), p(0x2000), p(0x3000), 128, 128, 96, 1, 1, p(0x4000), ws, None) \
+        == E.NVFP4_ERR_SHAPE
+    assert lib.nvfp4_linear_fwd(p(0x1000), p(0x2000), p(0x3000), 128, 128, 128, 1, 1, p(0x4000), ws - 1,
+                                None) == E.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_linear_fwd(None, p(0x2000), p(0x3000), 128, 128, 128, 1, 1, p(0x4000), ws, None) \
+        == E.NVFP4_ERR_INVALID_ARG
+    assert lib.nvfp4_linear_bwd(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), 100, 128, 128, 1, 1,
+                                1, p(0x6000), ws, None) == E.NVFP4_ERR_SHAPE
+    assert lib.nvfp4_relu2_fwd(p(0x1001), p(0x2000), 16, None) == E.NVFP4_ERR_ALIGNMENT
+    assert lib.nvfp4_relu2_bwd(None, p(0x2000), p(0x3000), 16, None) == E.NVFP4_ERR_INVALID_ARG

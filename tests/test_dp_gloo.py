@@ -1,0 +1,47 @@
+"""The data-parallel plumbing (gradient all-reduce, max-over-ranks timing,
+shard seeds) with two gloo ranks on CPU."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    from nvfp4_bit_precision_quantize_b200 import dp
+    dp.init("gloo", timeout_s=60)
+    g1 = torch.full((4, 3), float(rank + 1))
+    g2 = torch.arange(6, dtype=torch.float32) * (rank + 1)
+    dp.allreduce_grads([g1, g2])
+    slowest = dp.max_over_ranks(1.5 + rank)
+    seeds = dp.shard_seed(5, rank)
+    dp.barrier()
+    q.put((rank, g1.tolist(), g2.tolist(), slowest, seeds))
+    dp.finish()
+
+
+def test_two_rank_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, g1, g2, slowest, seed in res:
+        assert g1 == [[3.0] * 3] * 4
+        assert g2 == [float(3 * i) for i in range(6)]
+        assert slowest == 2.5
+    assert res[0][4] != res[1][4]
