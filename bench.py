@@ -252,7 +252,7 @@ def oracle_sample(budget_s=12.0):
     rng = np.random.default_rng(0)
     t_all = time.perf_counter()
     # quantiser: per-element cost of each mode on a 256 x 5120 bf16 slice (amax + quantise)
-    x = W.bf16_bits(W.normal(rng, (256, 5120)))
+    x = W.bf16_bits(W.normal(rng, (2048, 5120)))
     per_elem = {}
     for mode in [(False, False, False), (True, False, False), (True, True, True), (True, False, True)]:
         t0 = time.perf_counter()
@@ -271,7 +271,7 @@ def oracle_sample(budget_s=12.0):
                                                                              dtype=np.uint8), 1.0)
         b = (rng.integers(0, 256, (64, K // 2), dtype=np.uint8), rng.integers(0x20, 0x50, (64, K // 16),
                                                                              dtype=np.uint8), 1.0)
-        n = 96
+        n = 2560
         ms, ns = rng.integers(0, 64, n), rng.integers(0, 64, n)
         t0 = time.perf_counter()
         oracle.gemm_sampled(a, b, ms, ns)
@@ -279,15 +279,15 @@ def oracle_sample(budget_s=12.0):
         macs_done += n * K
         gemm_s += dt / (n * K) * (reps * M_TOK * HID * FFN)
     # relu^2 pair
-    y = W.bf16_bits(W.normal(rng, (1 << 20,)))
+    y = W.bf16_bits(W.normal(rng, (1 << 23,)))
     t0 = time.perf_counter()
     oracle.relu2_fwd(y)
     oracle.relu2_bwd(y, y)
     relu_s = (time.perf_counter() - t0) / y.size * n_h
     est = quant_s + gemm_s + relu_s
-    desc = ("oracle (plain C, 1 thread) on a bounded sample: 4 quantise modes on a 256x5120 bf16 slice, "
-            "%d FP64 sampled GEMM outputs (K = 5120/20480/8192), relu^2 on 2^20 elements; extrapolated "
-            "to the full step (%.1f s measured)" % (3 * 96, time.perf_counter() - t_all))
+    desc = ("oracle (plain C, 1 thread) on a bounded sample: 4 quantise modes on a 2048x5120 bf16 slice, "
+            "%d FP64 sampled GEMM outputs (K = 5120/20480/8192), relu^2 on 2^23 elements; extrapolated "
+            "to the full step (%.1f s measured)" % (3 * 2560, time.perf_counter() - t_all))
     return est, desc
 
 
@@ -426,8 +426,8 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
