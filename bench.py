@@ -423,6 +423,46 @@ def run_ours(args):
     dp.finish()
 
 
+def run_profile_case(case):
+    """A few calls of one kernel at a full workload size, for ncu captures (untimed)."""
+    from nvfp4_bit_precision_quantize_b200 import binding as B
+    from nvfp4_bit_precision_quantize_b200 import build as lib_build
+    lib_build.build()
+    B.load()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    rng = np.random.default_rng(7)
+    if case == "gemm":  # Fprop shape, random NVFP4 operands, bf16 out
+        def operand(rows, k):
+            return B.NVFP4Tensor(
+                codes=torch.randint(0, 256, (rows, k // 2), dtype=torch.uint8, device=dev, generator=g),
+                scales=torch.randint(0x20, 0x50, (B.nvfp4_scales_bytes(rows, k),), dtype=torch.uint8, device=dev,
+                                     generator=g),
+                tensor_scale=torch.ones(1, device=dev), rows=rows, k=k)
+        a, b = operand(M_TOK, HID), operand(FFN, HID)
+        out = torch.empty((M_TOK, FFN), dtype=torch.bfloat16, device=dev)
+        ws = B.workspace(256, dev)
+        for _ in range(3):
+            B.nvfp4_gemm(a, b, out=out, ws=ws)
+        B.nvfp4_check(ws)
+    elif case in ("quant_x", "quant_dy"):
+        if case == "quant_x":  # Fprop activation, rowwise RTN
+            x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, HID)))).to(dev)
+            kw = dict(orientation=B.NVFP4_ROWWISE)
+        else:  # Wgrad gradient operand: colwise, RHT + SR
+            x = W.bits_to_torch_bf16(W.bf16_bits(W.heavy_rows(rng, (2 * M_TOK, FFN), 1e-3, 2))).to(dev)
+            kw = dict(orientation=B.NVFP4_COLWISE, rounding=B.NVFP4_SR, rht=True)
+        ws = B.workspace(B.nvfp4_quantize_workspace_size(), dev)
+        q = None
+        for _ in range(3):
+            q = B.nvfp4_quantize(x, out=q, ws=ws, seed=SEED, **kw)
+    else:
+        raise SystemExit("unknown profile case " + case)
+    torch.cuda.synchronize()
+    print("profile case %s ok" % case)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,7 +470,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy"],
+                    help="run one kernel a few times for an ncu capture instead of the benchmark")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
