@@ -160,6 +160,30 @@ NVFP4_API nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const voi
                               void *workspace, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * nvfp4_linear_fwd_noalloc -- nvfp4_linear_fwd for callers that cannot
+ * allocate device memory (for instance code inside a framework that owns all
+ * device memory through its own pool, or a latency-critical loop that cannot
+ * afford the synchronisation of cudaMalloc/cudaFree).  The pages have no
+ * counterpart of this call: it only changes where the scratch lives.
+ * Same arguments, checks and result as nvfp4_linear_fwd, without a workspace:
+ * the scratch (status word, amax partials, both quantised operands) is one
+ * fixed device buffer of NVFP4_NOALLOC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits.  Calls
+ * whose nvfp4_linear_workspace_size(M, N, K) exceeds it return
+ * NVFP4_ERR_WORKSPACE and launch nothing.  The first call on a device looks
+ * the buffer's address up (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  The call allocates and
+ * frees nothing.  All calls share the one buffer and each starts by zeroing
+ * its status word: calls that overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.  A device-side
+ * timeout is recorded only in that shared buffer, which no public call reads.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+NVFP4_API nvfp4_status nvfp4_linear_fwd_noalloc(const void *X, const void *W, void *Y, int64_t M, int64_t N,
+                                                int64_t K, nvfp4_dtype dtype, nvfp4_dtype y_dtype,
+                                                cudaStream_t stream);
+
+/*
  * Squared-ReLU activation of the MLP block and its derivative, bf16 in/out,
  * n elements, contiguous, 16-byte aligned:
  *   h  = relu(y) * relu(y)          (binary32, then bf16 round-to-nearest-even)

@@ -33,7 +33,7 @@ NVFP4_SR = 1
 EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_size", "nvfp4_quantize",
            "nvfp4_gemm", "nvfp4_linear_workspace_size", "nvfp4_linear_fwd", "nvfp4_linear_bwd",
            "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
-           "nvfp4_status_string")
+           "nvfp4_status_string", "nvfp4_linear_fwd_noalloc")
 
 
 class CTensor(C.Structure):
@@ -74,6 +74,7 @@ def load():
         "nvfp4_check": (i32, [vp, vp]),
         "nvfp4_last_launch_count": (i32, []),
         "nvfp4_status_string": (C.c_char_p, [i32]),
+        "nvfp4_linear_fwd_noalloc": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -201,6 +202,19 @@ def nvfp4_linear_bwd(dY, X, W, seed=1234, dx_dtype=torch.bfloat16, dX=None, dW=N
                                  _dtype_code(dX.dtype), seed, _ptr(ws), ws.numel(), _stream(stream))
     _ok(st, "nvfp4_linear_bwd")
     return dX, dW
+
+
+def nvfp4_linear_fwd_noalloc(X, W, y_dtype=torch.bfloat16, out=None, stream=None):
+    """nvfp4_linear_fwd without a workspace: the library's fixed scratch buffer is
+    used instead (see include/nvfp4.h).  Only `out` may be allocated here, and only
+    when the caller passes none."""
+    M, K = X.shape
+    N = W.shape[0]
+    out = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
+    st = load().nvfp4_linear_fwd_noalloc(_ptr(X), _ptr(W), _ptr(out), M, N, K, _dtype_code(X.dtype),
+                                         _dtype_code(out.dtype), _stream(stream))
+    _ok(st, "nvfp4_linear_fwd_noalloc")
+    return out
 
 
 def nvfp4_relu2_fwd(y, out=None, stream=None):
