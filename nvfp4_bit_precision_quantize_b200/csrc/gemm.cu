@@ -7,20 +7,31 @@
 // section "Was konkret passiert ist"; format: aisight.pl, section
 // "Architektura NVFP4 kontra ograniczenia mikroskalowania".
 //
-// One CTA computes one 128 x 256 tile with warp roles:
-//   warp 0 (one lane)  producer: TMA loads of the code tiles (128-byte swizzle)
-//                      and bulk copies of the scale atoms into a 4-stage ring;
-//   warp 1             allocates TMEM; one lane copies each stage's scales into
-//                      TMEM (tcgen05.cp) and issues tcgen05.mma
-//                      kind::mxf4nvf4 block16 (K = 64 per instruction) with the
-//                      FP32 accumulator in TMEM; tcgen05.commit frees the stage;
+// Persistent kernel on CTA pairs (cluster of 2 SMs).  A pair owns a 256 x 256
+// output tile at a time: CTA rank r holds A rows [128r, 128r+128) of the tile
+// and B rows [128r, 128r+128), and the pair's tensor cores run one
+// M=256, N=256, K=64 tcgen05.mma (cta_group::2) per 64-k step, each CTA's
+// 128 x 256 FP32 accumulator in its own TMEM.  Warp roles, per CTA:
+//   warp 0 (one lane)  producer: TMA loads of this CTA's A and B code tiles
+//                      (128-byte swizzle) and scale atoms (A: its 128 rows;
+//                      B: all 256 rows) into a 5-stage ring; completion bytes
+//                      of both CTAs are counted on the leader's barrier;
+//   warp 1             allocates TMEM (pair-wide); on the leader one lane
+//                      copies each stage's scales into TMEM (tcgen05.cp,
+//                      cta_group::2) and issues the MMAs; tcgen05.commit
+//                      multicast to both CTAs frees the stage;
 //   warps 2..5         epilogue: tcgen05.ld of the accumulator (each warp its
-//                      32-lane TMEM quarter), scale by sA*sB, store f32 / bf16.
-// Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the CTA
-// records NVFP4_ERR_DEVICE_TIMEOUT in the status word, drains its own copies
-// and MMAs, frees TMEM and returns.  No TMA multicast is used.
+//                      32-lane TMEM quarter), hand TMEM back to the leader,
+//                      scale by sA*sB, store f32 / bf16.
+// Tiles are visited in groups of 8 tile columns so that the pairs running at
+// the same time share A and B panels in L2.  Every mbarrier wait is bounded
+// (about 2 s of %globaltimer); on expiry the CTA records
+// NVFP4_ERR_DEVICE_TIMEOUT in the status word, drains its copies and MMAs,
+// frees TMEM and returns.  No TMA load uses cluster multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -28,25 +39,27 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 256;           // BK in elements (128 bytes of codes)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK / 2;                   // 16 KB
-constexpr int B_BYTES = BN * BK / 2;                   // 32 KB
-constexpr int SFA_BYTES = (BM / 128) * (BK / 64) * 512;  // 2 KB
-constexpr int SFB_BYTES = (BN / 128) * (BK / 64) * 512;  // 4 KB
+constexpr int BM = 256, BN = 256, BK = 256;   // pair tile; BK in elements (128 bytes of codes)
+constexpr int STAGES = 5;
+constexpr int A_BYTES = 128 * BK / 2;          // 16 KB: this CTA's 128 A rows
+constexpr int B_BYTES = 128 * BK / 2;          // 16 KB: this CTA's 128 B rows
+constexpr int SFA_BYTES = (BK / 64) * 512;     // 2 KB: scale atoms of this CTA's A rows
+constexpr int SFB_BYTES = 2 * (BK / 64) * 512; // 4 KB: scale atoms of all 256 B rows
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;                    // acc 256 + SFA 16 + SFB 32, rounded up
-constexpr uint32_t TMEM_SFA = 256, TMEM_SFB = 272;
+constexpr uint32_t TMEM_COLS = 512;            // accumulator 256 columns + scales 48 columns, rounded up
+constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-constexpr int kTimeoutStatus = 7;                      // NVFP4_ERR_DEVICE_TIMEOUT
+constexpr uint64_t DRAIN_LIMIT_NS = 20000000ull;
+constexpr int kTimeoutStatus = 7;              // NVFP4_ERR_DEVICE_TIMEOUT
+constexpr int GROUP_N = 8;                     // tile columns per raster group
 
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1) at bits 7-9 /
 // 10-12, K-major, N >> 3 at bits 17-22, UE4M3 scales (bit 23 = 0), M >> 4 at
-// bits 24-28, scale-factor byte ids 0, dense K = 64.
+// bits 24-28 (M = 256 across the pair), scale-factor byte ids 0, dense K = 64.
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -57,26 +70,53 @@ __device__ __forceinline__ uint64_t globaltimer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+__device__ __forceinline__ uint32_t cta_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t nclusters_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false once the limit passes or another role has given up.
+// Bounded wait: false once the limit passes or another role of this CTA has given up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          bool honour_abort = true) {
+                                          bool honour_abort = true, uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
@@ -84,40 +124,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         for (int i = 0; i < 16; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (honour_abort && *abort_flag) return false;
-        if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             return false;
         }
     }
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+// Tile load into this CTA's shared memory whose completion bytes are counted
+// on the leader's barrier (a shared::cluster address).
+__device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap *map, uint32_t leader_bar, int x, int y,
+                                              uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(dst),
-        "l"(map), "r"(bar), "r"(x), "r"(y)
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(map), "r"(leader_bar), "r"(x), "r"(y), "l"(policy)
         : "memory");
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+// Arrives on the barrier at the same offset in both CTAs once every MMA issued so far has completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
 }
-// Scale atom (32 rows x 16 bytes in smem) -> 32 TMEM lanes x 4 columns, copied to all four lane quarters.
+__device__ __forceinline__ void tc_commit_self(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// Scale atom (32 rows x 16 bytes in smem) -> 32 TMEM lanes x 4 columns, copied to
+// all four lane quarters, in both CTAs of the pair (each from its own smem).
 __device__ __forceinline__ void tc_cp_scales(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa, uint32_t sfb, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
         "l"(a), "l"(b), "r"(IDESC), "r"(acc), "r"(sfa), "r"(sfb)
         : "memory");
 }
@@ -131,6 +177,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_global_v4(void *dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                             uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(a), "r"(b), "r"(c),
+                 "r"(d), "l"(policy)
+                 : "memory");
 }
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes,
@@ -146,130 +198,223 @@ __device__ __forceinline__ uint64_t sdesc_scales(uint32_t saddr) {
 }
 
 struct KParams {
-    const uint8_t *sfa, *sfb;
     const float *tsa, *tsb;
     void *C;
     int64_t ldc;
     int M, N, K;
-    int kb4;          // scale atoms per 128-row tile (= ceil(K / 64))
-    int b_rowtiles;   // 128-row tiles of B's scale buffer (= ceil(N / 128))
+    int kb4;  // scale atoms per 128-row tile (= K / 64)
     int c_bf16;
+    int tiles_m, tiles_n, num_tiles;
     int *status;
 };
 
-__global__ void __launch_bounds__(THREADS, 1)
+// Tile t -> (tile row, tile column).  Tile columns form bands of GROUP_N; inside
+// a band, consecutive t walk along a tile row, then down to the next tile row.
+__device__ __forceinline__ void tile_coords(const KParams &p, int t, int &mt, int &nt) {
+    const int per_group = p.tiles_m * GROUP_N;
+    const int g = t / per_group, r = t - g * per_group;
+    const int gw = min(GROUP_N, p.tiles_n - g * GROUP_N);
+    mt = r / gw;
+    nt = g * GROUP_N + (r - mt * gw);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                       const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    const uint32_t bar_full = smem_u32(bars);                // [S] leader: both CTAs' bytes of a stage
+    const uint32_t bar_empty = smem_u32(bars + STAGES);      // [S] each CTA: MMAs reading the stage done
+    const uint32_t bar_accf = smem_u32(bars + 2 * STAGES);   // each CTA: accumulator complete
+    const uint32_t bar_acce = smem_u32(bars + 2 * STAGES + 1);  // leader: accumulator read (8 epilogue warps)
+    const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2); // leader: every MMA done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    const uint32_t bar_full = smem_u32(bars), bar_empty = smem_u32(bars + STAGES),
-                   bar_acc = smem_u32(bars + 2 * STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
-    const int num_kt = (p.K + BK - 1) / BK;
+    const uint32_t rank = cta_rank();
+    const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+    const int num_kt = p.K / BK + ((p.K % BK) ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        mbar_init(bar_acc, 1);
+        mbar_init(bar_accf, 1);
+        mbar_init(bar_acce, 8);
+        mbar_init(bar_drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
         __syncwarp();
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(TMEM_COLS)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t smem_base = smem_u32(smem);
 
-    if (warp == 0 && lane == 0) {
-        // ---------------- producer ----------------
-        int issued = 0;
-        for (int kt = 0; kt < num_kt; ++kt) {
-            const int s = kt % STAGES;
-            const uint32_t ph = (kt / STAGES) & 1;
-            if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag)) break;
-            const int steps = min(BK / 64, (p.K - kt * BK) / 64);
-            const int b_tiles = min(2, p.b_rowtiles - 2 * (int)blockIdx.x);
-            const uint32_t bytes = A_BYTES + B_BYTES + steps * 512 * (1 + b_tiles);
-            uint8_t *st = smem + s * STAGE_BYTES;
-            const uint32_t fb = bar_full + 8 * s;
-            mbar_expect_tx(fb, bytes);
-            tma_load_2d(smem_u32(st), &map_a, fb, kt * (BK / 2), m0);
-            tma_load_2d(smem_u32(st + A_BYTES), &map_b, fb, kt * (BK / 2), n0);
-            bulk_load(smem_u32(st + A_BYTES + B_BYTES),
-                      p.sfa + ((size_t)blockIdx.y * p.kb4 + (size_t)kt * 4) * 512, steps * 512, fb);
-            for (int t = 0; t < b_tiles; ++t)
-                bulk_load(smem_u32(st + A_BYTES + B_BYTES + SFA_BYTES + t * 2048),
-                          p.sfb + ((size_t)(2 * blockIdx.x + t) * p.kb4 + (size_t)kt * 4) * 512, steps * 512, fb);
-            issued = kt + 1;
-        }
-        // Drain: every issued stage must have landed before the CTA may exit.
-        for (int kt = max(0, issued - STAGES); kt < issued; ++kt)
-            mbar_wait(bar_full + 8 * (kt % STAGES), (kt / STAGES) & 1, abort_flag, false);
-    } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer ----------------
-        for (int kt = 0; kt < num_kt; ++kt) {
-            const int s = kt % STAGES;
-            const uint32_t ph = (kt / STAGES) & 1;
-            if (!mbar_wait(bar_full + 8 * s, ph, abort_flag)) break;
-            tc_fence_after();
-            const int steps = min(BK / 64, (p.K - kt * BK) / 64);
-            const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-            const uint32_t sb = sa + A_BYTES, ssfa = sb + B_BYTES, ssfb = ssfa + SFA_BYTES;
-            for (int j = 0; j < steps; ++j) {
-                tc_cp_scales(tmem + TMEM_SFA + 4 * j, sdesc_scales(ssfa + 512 * j));
-                tc_cp_scales(tmem + TMEM_SFB + 8 * j, sdesc_scales(ssfb + 512 * j));
-                tc_cp_scales(tmem + TMEM_SFB + 8 * j + 4, sdesc_scales(ssfb + 2048 + 512 * j));
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer (both CTAs) ----------------
+            uint64_t policy;
+            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
+            int it = 0;
+            bool ok = true;
+            for (int t = cid; t < p.num_tiles && ok; t += ncl) {
+                int mt, nt;
+                tile_coords(p, t, mt, nt);
+                const int m0 = mt * BM + 128 * (int)rank, n0 = nt * BN;
+                for (int kt = 0; kt < num_kt; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(bar_empty + 8 * s, ((it / STAGES) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = smem_base + s * STAGE_BYTES;
+                    const uint32_t full_leader = mapa(bar_full + 8 * s, 0);
+                    // Out-of-range rows, columns and atoms are zero-filled and still
+                    // counted, so every stage brings exactly STAGE_BYTES per CTA.
+                    if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_BYTES);
+                    tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
+                    tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, (m0 / 128) * p.kb4 + kt * 4,
+                                  policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0,
+                                  (n0 / 128) * p.kb4 + kt * 4, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES + 2048, &map_sfb, full_leader, 0,
+                                  (n0 / 128 + 1) * p.kb4 + kt * 4, policy);
+                }
             }
-            const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sb);
-            for (int j = 0; j < steps; ++j)
-                tc_mma(tmem, da + 2 * j, db + 2 * j, tmem + TMEM_SFA + 4 * j, tmem + TMEM_SFB + 8 * j,
-                       (kt > 0 || j > 0) ? 1u : 0u);
-            tc_commit(bar_empty + 8 * s);
+            // This CTA's loads complete on the leader's barriers; the leader drains them.
         }
-        tc_commit(bar_acc);  // arrives once every MMA issued above has completed
-    } else if (warp >= 2) {
-        // ---------------- epilogue ----------------
-        const int quarter = warp & 3;
-        bool ok = mbar_wait(bar_acc, 0, abort_flag, false);
-        ok = __all_sync(0xFFFFFFFFu, ok) && !*abort_flag;
-        tc_fence_after();
-        if (ok) {
-            const float scale = __fmul_rn(*p.tsa, *p.tsb);
-            const int row = m0 + quarter * 32 + lane;
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (leader only) ----------------
+            int it = 0, tile_i = 0;
+            bool ok = true;
+            for (int t = cid; t < p.num_tiles && ok; t += ncl, ++tile_i) {
+                if (!mbar_wait(bar_acce, (tile_i & 1) ^ 1, abort_flag)) break;
+                tc_fence_after();
+                for (int kt = 0; kt < num_kt; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    // The barrier's completion makes the TMA writes visible to the tensor cores.
+                    if (!mbar_wait(bar_full + 8 * s, (it / STAGES) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = smem_base + s * STAGE_BYTES;
+                    const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + A_BYTES);
+                    const uint64_t dsa = sdesc_scales(sa + A_BYTES + B_BYTES);
+                    const uint64_t dsb = sdesc_scales(sa + A_BYTES + B_BYTES + SFA_BYTES);
+                    const uint32_t sf = tmem + TMEM_SF;
+                    // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
+                    // +128 for B's second 128-row tile, +2 per 64-k step of codes.
+                    if (kt * BK + BK <= p.K) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            tc_cp_scales(sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    } else {
+                        const int steps = (p.K - kt * BK) / 64;
+                        for (int j = 0; j < steps; ++j) {
+                            tc_cp_scales(sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                        }
+                        for (int j = 0; j < steps; ++j)
+                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(bar_empty + 8 * s);
+                }
+                if (ok) tc_commit_pair(bar_accf);
+            }
+            tc_commit_self(bar_drain);
+            mbar_wait(bar_drain, 0, abort_flag, false);
+            if (*abort_flag) {
+                // Stages the producers may still be filling: wait (briefly) for their bytes.
+                for (int k = it; k < it + STAGES; ++k)
+                    mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
+            }
+        }
+    } else {
+        // ---------------- epilogue (both CTAs) ----------------
+        const uint32_t q = warp & 3;
+        const uint32_t lane_base = (q * 32u) << 16;
+        uint64_t policy;
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+        const float scale = __fmul_rn(*p.tsa, *p.tsb);
+        int tile_i = 0;
+        for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
+            bool ok = mbar_wait(bar_accf, tile_i & 1, abort_flag);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            int mt, nt;
+            tile_coords(p, t, mt, nt);
+            const int row = mt * BM + 128 * (int)rank + (int)q * 32 + lane;
             const bool row_ok = row < p.M;
+            const int n0 = nt * BN;
+            if (p.c_bf16 && n0 + BN <= p.N) {
+                // Full-width bf16 tile: the whole accumulator row fits in registers
+                // as packed pairs, so TMEM is handed back before any store.
+                uint32_t w[BN / 2];
+#pragma unroll
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + ch * 32, r);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
+                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[ch * 16 + j]) : "f"(hi), "f"(lo));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
+                if (!row_ok) continue;
+                uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + n0;
+#pragma unroll
+                for (int j = 0; j < BN / 8; ++j) st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
+                continue;
+            }
 #pragma unroll 1
             for (int ch = 0; ch < BN / 32; ++ch) {
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + ch * 32, r);
+                tmem_ld32(tmem + lane_base + ch * 32, r);
+                if (ch == BN / 32 - 1) {  // accumulator fully read: hand TMEM back to the MMA issuer
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
+                }
                 const int col0 = n0 + ch * 32;
                 if (!row_ok || col0 >= p.N) continue;
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[j]), scale);
                 if (p.c_bf16) {
                     uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + col0;
                     uint32_t w[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[j]) : "f"(v[2 * j + 1]), "f"(v[2 * j]));
+                    for (int j = 0; j < 16; ++j) {
+                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
+                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[j]) : "f"(hi), "f"(lo));
+                    }
                     if (col0 + 32 <= p.N) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            reinterpret_cast<uint4 *>(dst)[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                        for (int j = 0; j < 4; ++j) st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
@@ -277,10 +422,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 } else {
                     float *dst = static_cast<float *>(p.C) + (int64_t)row * p.ldc + col0;
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[j]), scale);
                     if (col0 + 32 <= p.N) {
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            reinterpret_cast<float4 *>(dst)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                            st_global_v4(dst + 4 * j, __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                                         __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]), policy);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
@@ -292,11 +441,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
     if (threadIdx.x == 0 && *abort_flag && p.status) atomicExch(p.status, kTimeoutStatus);
 }
@@ -314,16 +463,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D byte view of a codes buffer: [rows x K/2], box = 128 bytes x box_rows, 128B swizzle.
-bool make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_t K, uint32_t box_rows) {
+// 2-D byte view of a codes buffer: [rows x K/2], box = 128 bytes x 128 rows, 128B swizzle.
+bool make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_t K) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t box[2] = {128u, 128u};
     cuuint32_t estr[2] = {1u, 1u};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A scale buffer as rows of one 512-byte atom (128 words): [atoms x 128] words,
+// box = 4 atoms (one 256-k stage of one 128-row tile).
+bool make_scale_map(CUtensorMap *map, const uint8_t *scales, int64_t rows, int64_t K) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int64_t atoms = ((rows + 127) / 128) * (K / 64);
+    cuuint64_t dims[2] = {128u, (cuuint64_t)atoms};
+    cuuint64_t strides[1] = {512u};
+    cuuint32_t box[2] = {128u, 4u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -336,22 +500,32 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
         ++*launches;
         return cudaMemset2DAsync(a.C, (size_t)a.ldc * esz, 0, (size_t)a.N * esz, (size_t)a.M, s);
     }
-    CUtensorMap map_a, map_b;
-    if (!make_codes_map(&map_a, a.a_codes, a.M, a.K, BM) || !make_codes_map(&map_b, a.b_codes, a.N, a.K, BN))
+    CUtensorMap map_a, map_b, map_sfa, map_sfb;
+    if (!make_codes_map(&map_a, a.a_codes, a.M, a.K) || !make_codes_map(&map_b, a.b_codes, a.N, a.K) ||
+        !make_scale_map(&map_sfa, a.a_scales, a.M, a.K) || !make_scale_map(&map_sfb, a.b_scales, a.N, a.K))
         return cudaErrorInvalidValue;
-    static bool configured[64] = {};
+    constexpr int kMaxDev = 64;
+    static int max_clusters[kMaxDev] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    if (!max_clusters[dev]) {
         e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        configured[dev] = true;
+        // Pairs that can be resident at once (one CTA per SM).
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = num_sms() / 2;
+        }
+        max_clusters[dev] = n;
     }
     KParams p;
-    p.sfa = a.a_scales;
-    p.sfb = a.b_scales;
     p.tsa = a.a_ts;
     p.tsb = a.b_ts;
     p.C = a.C;
@@ -359,12 +533,14 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.M = (int)a.M;
     p.N = (int)a.N;
     p.K = (int)a.K;
-    p.kb4 = (int)((a.K + 63) / 64);
-    p.b_rowtiles = (int)((a.N + 127) / 128);
+    p.kb4 = (int)(a.K / 64);
     p.c_bf16 = a.c_bf16 ? 1 : 0;
+    p.tiles_m = (int)((a.M + BM - 1) / BM);
+    p.tiles_n = (int)((a.N + BN - 1) / BN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
     p.status = a.status;
-    dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + BM - 1) / BM));
-    gemm_nvfp4_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(map_a, map_b, p);
+    const int pairs = std::min(p.num_tiles, max_clusters[dev]);
+    gemm_nvfp4_kernel<<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, p);
     ++*launches;
     return cudaGetLastError();
 }
