@@ -20,9 +20,10 @@
 //                      copies each stage's scales into TMEM (tcgen05.cp,
 //                      cta_group::2) and issues the MMAs; tcgen05.commit
 //                      multicast to both CTAs frees the stage;
-//   warps 2..5         epilogue: tcgen05.ld of the accumulator (each warp its
-//                      32-lane TMEM quarter), hand TMEM back to the leader,
-//                      scale by sA*sB, store f32 / bf16.
+//   warps 2..9         epilogue: two warps per 32-lane TMEM quarter, each
+//                      reading 128 accumulator columns into registers
+//                      (tcgen05.ld), then handing TMEM back to the leader
+//                      before it scales by sA*sB and stores f32 / bf16.
 // Tiles are visited in groups of 8 tile columns so that the pairs running at
 // the same time share A and B panels in L2.  Every mbarrier wait is bounded
 // (about 2 s of %globaltimer); on expiry the CTA records
@@ -49,7 +50,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;                    // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;            // accumulator 256 columns + scales 48 columns, rounded up
 constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
@@ -114,10 +116,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false once the limit passes or another role of this CTA has given up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          bool honour_abort = true, uint64_t limit_ns = WAIT_LIMIT_NS) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait, slow path: false once the limit passes or another role of this
+// CTA has given up.  Kept out of line so the issue loops stay short.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, bool honour_abort,
+                                            uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (;;) {
 #pragma unroll 1
@@ -129,6 +131,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          bool honour_abort = true, uint64_t limit_ns = WAIT_LIMIT_NS) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort_flag, honour_abort, limit_ns);
 }
 
 // Tile load into this CTA's shared memory whose completion bytes are counted
@@ -202,7 +209,9 @@ struct KParams {
     void *C;
     int64_t ldc;
     int M, N, K;
-    int kb4;  // scale atoms per 128-row tile (= K / 64)
+    int kb4;    // scale atoms per 128-row tile (= K / 64)
+    int kfull;  // full 256-k stages (= K / 256)
+    int ktail;  // 64-k steps in a last, partial stage (= (K % 256) / 64)
     int c_bf16;
     int tiles_m, tiles_n, num_tiles;
     int *status;
@@ -236,7 +245,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cta_rank();
     const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
-    const int num_kt = p.K / BK + ((p.K % BK) ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -244,7 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(bar_empty + 8 * s, 1);
         }
         mbar_init(bar_accf, 1);
-        mbar_init(bar_acce, 8);
+        mbar_init(bar_acce, 2 * EPI_WARPS);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -261,21 +269,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t smem_base = smem_u32(smem);
+    const int num_kt = p.kfull + (p.ktail ? 1 : 0);
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- producer (both CTAs) ----------------
             uint64_t policy;
             asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
-            int it = 0;
+            uint32_t s = 0, ph = 0;
             bool ok = true;
             for (int t = cid; t < p.num_tiles && ok; t += ncl) {
                 int mt, nt;
                 tile_coords(p, t, mt, nt);
                 const int m0 = mt * BM + 128 * (int)rank, n0 = nt * BN;
-                for (int kt = 0; kt < num_kt; ++kt, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(bar_empty + 8 * s, ((it / STAGES) & 1) ^ 1, abort_flag)) {
+                const int ya = (m0 / 128) * p.kb4, yb = (n0 / 128) * p.kb4;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -286,12 +295,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_BYTES);
                     tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
                     tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, (m0 / 128) * p.kb4 + kt * 4,
-                                  policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0,
-                                  (n0 / 128) * p.kb4 + kt * 4, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, ya + kt * 4, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * 4, policy);
                     tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES + 2048, &map_sfb, full_leader, 0,
-                                  (n0 / 128 + 1) * p.kb4 + kt * 4, policy);
+                                  yb + p.kb4 + kt * 4, policy);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
             }
             // This CTA's loads complete on the leader's barriers; the leader drains them.
@@ -299,15 +310,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ---------------- MMA issuer (leader only) ----------------
-            int it = 0, tile_i = 0;
+            const int kfull = p.kfull, ktail = p.ktail;
+            uint32_t s = 0, ph = 0;
+            int consumed = 0, tile_i = 0;
             bool ok = true;
-            for (int t = cid; t < p.num_tiles && ok; t += ncl, ++tile_i) {
-                if (!mbar_wait(bar_acce, (tile_i & 1) ^ 1, abort_flag)) break;
+            for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
+                if (!mbar_wait(bar_acce, (tile_i & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                for (int kt = 0; kt < num_kt; ++kt, ++it) {
-                    const int s = it % STAGES;
+                uint32_t acc = 0;  // the first MMA of a tile overwrites the accumulator
+                for (int kt = 0; kt < num_kt; ++kt) {
                     // The barrier's completion makes the TMA writes visible to the tensor cores.
-                    if (!mbar_wait(bar_full + 8 * s, (it / STAGES) & 1, abort_flag)) {
+                    if (!mbar_wait(bar_full + 8 * s, ph, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -318,42 +334,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t sf = tmem + TMEM_SF;
                     // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
                     // +128 for B's second 128-row tile, +2 per 64-k step of codes.
-                    if (kt * BK + BK <= p.K) {
+                    if (kt < kfull) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             tc_cp_scales(sf + 4 * j, dsa + 32 * j);
                             tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
                             tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
+                        tc_mma(tmem, da, db, sf, sf + 16, acc);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                        for (int j = 1; j < 4; ++j) tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
                     } else {
-                        const int steps = (p.K - kt * BK) / 64;
-                        for (int j = 0; j < steps; ++j) {
+                        for (int j = 0; j < ktail; ++j) {
                             tc_cp_scales(sf + 4 * j, dsa + 32 * j);
                             tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
                             tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
-                        for (int j = 0; j < steps; ++j)
-                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                        for (int j = 0; j < ktail; ++j)
+                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (acc | (uint32_t)j) ? 1u : 0u);
                     }
+                    acc = 1;
                     tc_commit_pair(bar_empty + 8 * s);
+                    ++consumed;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
-                if (ok) tc_commit_pair(bar_accf);
+                if (!ok) break;
+                tc_commit_pair(bar_accf);
             }
             tc_commit_self(bar_drain);
             mbar_wait(bar_drain, 0, abort_flag, false);
             if (*abort_flag) {
                 // Stages the producers may still be filling: wait (briefly) for their bytes.
-                for (int k = it; k < it + STAGES; ++k)
+                for (int k = consumed; k < consumed + STAGES; ++k)
                     mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
             }
         }
     } else {
         // ---------------- epilogue (both CTAs) ----------------
+        // Warp w reads TMEM lane quarter w % 4 (the quarter a warp may access) and
+        // columns [128 h, 128 h + 128) of the accumulator, h = (w - 2) / 4.
         const uint32_t q = warp & 3;
-        const uint32_t lane_base = (q * 32u) << 16;
+        const int h = (warp - 2) >> 2;
+        const uint32_t tbase = tmem + ((q * 32u) << 16) + 128u * (uint32_t)h;
         uint64_t policy;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
         const float scale = __fmul_rn(*p.tsa, *p.tsb);
@@ -367,41 +392,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tile_coords(p, t, mt, nt);
             const int row = mt * BM + 128 * (int)rank + (int)q * 32 + lane;
             const bool row_ok = row < p.M;
-            const int n0 = nt * BN;
-            if (p.c_bf16 && n0 + BN <= p.N) {
-                // Full-width bf16 tile: the whole accumulator row fits in registers
-                // as packed pairs, so TMEM is handed back before any store.
-                uint32_t w[BN / 2];
+            const int c0 = nt * BN + 128 * h;  // first column of this warp's half
+            if (c0 + 128 <= p.N) {
+                // The warp's whole half-row fits in registers: read all of it, hand
+                // TMEM back, then scale and store.
+                if (p.c_bf16) {
+                    uint32_t w[64];
 #pragma unroll
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + ch * 32, r);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld32(tbase + ch * 32, r);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
-                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[ch * 16 + j]) : "f"(hi), "f"(lo));
+                        for (int j = 0; j < 16; ++j) {
+                            const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
+                            const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
+                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[ch * 16 + j]) : "f"(hi), "f"(lo));
+                        }
                     }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
-                if (!row_ok) continue;
-                uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + n0;
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
+                    if (!row_ok) continue;
+                    uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + c0;
 #pragma unroll
-                for (int j = 0; j < BN / 8; ++j) st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
+                    for (int j = 0; j < 16; ++j)
+                        st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
+                } else {
+                    uint32_t v[128];
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t r[32];
+                        tmem_ld32(tbase + ch * 32, r);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[ch * 32 + j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), scale));
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
+                    if (!row_ok) continue;
+                    float *dst = static_cast<float *>(p.C) + (int64_t)row * p.ldc + c0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) st_global_v4(dst + 4 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3], policy);
+                }
                 continue;
             }
+            // Ragged right edge: 32 columns at a time, TMEM released after the last read.
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
+            for (int ch = 0; ch < 4; ++ch) {
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_base + ch * 32, r);
-                if (ch == BN / 32 - 1) {  // accumulator fully read: hand TMEM back to the MMA issuer
+                tmem_ld32(tbase + ch * 32, r);
+                if (ch == 3) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
                 }
-                const int col0 = n0 + ch * 32;
+                const int col0 = c0 + ch * 32;
                 if (!row_ok || col0 >= p.N) continue;
                 if (p.c_bf16) {
                     uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + col0;
@@ -422,18 +467,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                 } else {
                     float *dst = static_cast<float *>(p.C) + (int64_t)row * p.ldc + col0;
-                    float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__uint_as_float(r[j]), scale);
+                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), scale));
                     if (col0 + 32 <= p.N) {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            st_global_v4(dst + 4 * j, __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                                         __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]), policy);
+                        for (int j = 0; j < 8; ++j) st_global_v4(dst + 4 * j, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3], policy);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) dst[j] = v[j];
+                            if (col0 + j < p.N) dst[j] = __uint_as_float(r[j]);
                     }
                 }
             }
@@ -534,6 +576,8 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.N = (int)a.N;
     p.K = (int)a.K;
     p.kb4 = (int)(a.K / 64);
+    p.kfull = (int)(a.K / BK);
+    p.ktail = (int)((a.K % BK) / 64);
     p.c_bf16 = a.c_bf16 ? 1 : 0;
     p.tiles_m = (int)((a.M + BM - 1) / BM);
     p.tiles_n = (int)((a.N + BN - 1) / BN);
