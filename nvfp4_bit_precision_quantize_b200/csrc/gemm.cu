@@ -16,10 +16,16 @@
 //                      (128-byte swizzle) and scale atoms (A: its 128 rows;
 //                      B: all 256 rows) into a 5-stage ring; completion bytes
 //                      of both CTAs are counted on the leader's barrier;
-//   warp 1             allocates TMEM (pair-wide); on the leader one lane
+//   warp 1             allocates TMEM (pair-wide); on the leader the whole
+//                      warp runs the issue loop and one lane, by predicate,
 //                      copies each stage's scales into TMEM (tcgen05.cp,
 //                      cta_group::2) and issues the MMAs; tcgen05.commit
 //                      multicast to both CTAs frees the stage;
+//   warp 10            waiter (leader): polls the stage-full and
+//                      accumulator-free barriers and relays each event to the
+//                      MMA warp through a hardware named barrier, so that the
+//                      issuing warp never waits on shared memory (its latency
+//                      is high while the tensor cores stream operands);
 //   warps 2..9         epilogue: two warps per 32-lane TMEM quarter, each
 //                      reading 128 accumulator columns into registers
 //                      (tcgen05.ld), then handing TMEM back to the leader
@@ -50,8 +56,12 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr int THREADS = 320;                    // producer, MMA, 8 epilogue warps
+constexpr int THREADS = 352;                    // producer, MMA, 8 epilogue warps, waiter
 constexpr int EPI_WARPS = 8;
+constexpr int WAITER_WARP = 10;
+// Hardware named barriers (64 threads: the waiter warp and the MMA warp).
+constexpr uint32_t NB_ACC = 1;     // accumulator free for the next tile
+constexpr uint32_t NB_STAGE0 = 2;  // NB_STAGE0 + s: stage s loaded
 constexpr uint32_t TMEM_COLS = 512;            // accumulator 256 columns + scales 48 columns, rounded up
 constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
@@ -109,6 +119,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// The same with cluster-scope acquire, for barriers that CTAs of the pair arrive on.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
@@ -116,6 +138,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ void named_sync(uint32_t id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
 // Bounded wait, slow path: false once the limit passes or another role of this
 // CTA has given up.  Kept out of line so the issue loops stay short.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, bool honour_abort,
@@ -151,28 +174,70 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap *m
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Arrives on the barrier at the same offset in both CTAs once every MMA issued so far has completed.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-        "h"((uint16_t)3)
-        : "memory");
-}
-__device__ __forceinline__ void tc_commit_self(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
+// The MMA warp runs its loop on all 32 lanes (no divergent branches around the
+// issue sequence) and issues each tensor-core instruction from the lanes whose
+// `issue` is non-zero -- one lane -- through a PTX predicate.
 // Scale atom (32 rows x 16 bytes in smem) -> 32 TMEM lanes x 4 columns, copied to
 // all four lane quarters, in both CTAs of the pair (each from its own smem).
-__device__ __forceinline__ void tc_cp_scales(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t sfa, uint32_t sfb, uint32_t acc) {
+__device__ __forceinline__ void tc_cp_scales_if(uint32_t issue, uint32_t taddr, uint64_t sdesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(IDESC), "r"(acc), "r"(sfa), "r"(sfb)
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t"
+        "@q tcgen05.cp.cta_group::2.32x128b.warpx4 [%1], %2;\n\t}" ::"r"(issue),
+        "r"(taddr), "l"(sdesc)
         : "memory");
+}
+__device__ __forceinline__ void tc_mma_if(uint32_t issue, uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
+                                          uint32_t sfb, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %7, 0;\n\t"
+        "@q tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(IDESC), "r"(acc), "r"(sfa), "r"(sfb), "r"(issue)
+        : "memory");
+}
+// Arrives on the barrier at the same offset in both CTAs once every MMA issued so far has completed.
+__device__ __forceinline__ void tc_commit_pair_if(uint32_t issue, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t"
+        "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%1], %2;\n\t}" ::"r"(
+            issue),
+        "r"(bar), "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_self_if(uint32_t issue, uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t"
+        "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%1];\n\t}" ::"r"(issue),
+        "r"(bar)
+        : "memory");
+}
+// Warp-uniform bounded wait: every lane returns the same answer.
+template <bool CLUSTER>
+__device__ __forceinline__ bool try_wait_scoped(uint32_t bar, uint32_t parity) {
+    return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+}
+template <bool CLUSTER>
+__device__ __noinline__ bool mbar_wait_warp_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                 bool honour_abort, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (__all_sync(0xFFFFFFFFu, try_wait_scoped<CLUSTER>(bar, parity))) return true;
+        const bool aborted = __any_sync(0xFFFFFFFFu, honour_abort && *abort_flag);
+        if (aborted) return false;
+        if (__any_sync(0xFFFFFFFFu, globaltimer() - t0 > limit_ns)) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                               bool honour_abort = true, uint64_t limit_ns = WAIT_LIMIT_NS) {
+    if (__all_sync(0xFFFFFFFFu, try_wait_scoped<CLUSTER>(bar, parity))) return true;
+    return mbar_wait_warp_slow<CLUSTER>(bar, parity, abort_flag, honour_abort, limit_ns);
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -241,6 +306,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2); // leader: every MMA done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *stop_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // waiter -> MMA warp, per tile
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cta_rank();
@@ -255,6 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mbar_init(bar_acce, 2 * EPI_WARPS);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
+        *stop_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -308,25 +375,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // This CTA's loads complete on the leader's barriers; the leader drains them.
         }
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
-            // ---------------- MMA issuer (leader only) ----------------
+        if (rank == 0) {
+            // ---------------- MMA issuer (leader's warp 1, lane 0 issues) ----------------
+            const uint32_t issue = lane == 0 ? 1u : 0u;
             const int kfull = p.kfull, ktail = p.ktail;
             uint32_t s = 0, ph = 0;
             int consumed = 0, tile_i = 0;
-            bool ok = true;
+            // Every event this warp waits for comes from the waiter warp through a
+            // named barrier: the loop below reads no shared memory per stage.
             for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
-                if (!mbar_wait(bar_acce, (tile_i & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                named_sync(NB_ACC);
+                if (*stop_flag) break;  // written by the waiter before the barrier
                 tc_fence_after();
                 uint32_t acc = 0;  // the first MMA of a tile overwrites the accumulator
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    // The barrier's completion makes the TMA writes visible to the tensor cores.
-                    if (!mbar_wait(bar_full + 8 * s, ph, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    // Stage s has landed (the waiter saw its barrier complete).
+                    named_sync(NB_STAGE0 + s);
                     const uint32_t sa = smem_base + s * STAGE_BYTES;
                     const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + A_BYTES);
                     const uint64_t dsa = sdesc_scales(sa + A_BYTES + B_BYTES);
@@ -334,42 +398,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t sf = tmem + TMEM_SF;
                     // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
                     // +128 for B's second 128-row tile, +2 per 64-k step of codes.
-                    if (kt < kfull) {
+                    const int steps = kt < kfull ? 4 : ktail;
+                    if (steps == 4) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            tc_cp_scales(sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
-                        tc_mma(tmem, da, db, sf, sf + 16, acc);
+                        tc_mma_if(issue, tmem, da, db, sf, sf + 16, acc);
 #pragma unroll
-                        for (int j = 1; j < 4; ++j) tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
+                        for (int j = 1; j < 4; ++j)
+                            tc_mma_if(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
                     } else {
-                        for (int j = 0; j < ktail; ++j) {
-                            tc_cp_scales(sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales(sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales(sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                        for (int j = 0; j < steps; ++j) {
+                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
-                        for (int j = 0; j < ktail; ++j)
-                            tc_mma(tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, (acc | (uint32_t)j) ? 1u : 0u);
+                        for (int j = 0; j < steps; ++j)
+                            tc_mma_if(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
+                                      (acc | (uint32_t)j) ? 1u : 0u);
                     }
                     acc = 1;
-                    tc_commit_pair(bar_empty + 8 * s);
+                    tc_commit_pair_if(issue, bar_empty + 8 * s);
                     ++consumed;
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
-                if (!ok) break;
-                tc_commit_pair(bar_accf);
+                tc_commit_pair_if(issue, bar_accf);
             }
-            tc_commit_self(bar_drain);
-            mbar_wait(bar_drain, 0, abort_flag, false);
+            tc_commit_self_if(issue, bar_drain);
+            mbar_wait_warp(bar_drain, 0, abort_flag, false);
             if (*abort_flag) {
                 // Stages the producers may still be filling: wait (briefly) for their bytes.
                 for (int k = consumed; k < consumed + STAGES; ++k)
-                    mbar_wait(bar_full + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
+                    mbar_wait_warp(bar_full + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
+            }
+        }
+    } else if (warp == WAITER_WARP) {
+        if (rank == 0) {
+            // ---------------- waiter (leader only) ----------------
+            // Waits on the accumulator-free and stage-full barriers in the order the
+            // MMA warp consumes them and relays each through a named barrier.  After
+            // a timeout inside a tile it keeps relaying without waiting until the
+            // tile ends, then both warps stop.
+            // Both warps take the same named barriers in the same order (bar.sync on
+            // both sides: neither can run ahead), and leave the tile loop together:
+            // the stop decision is written before the per-tile barrier and read by
+            // the MMA warp after it.
+            uint32_t s = 0, ph = 0;
+            int tile_i = 0;
+            bool ok = true;
+            for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
+                if (ok) ok = mbar_wait_warp<true>(bar_acce, (tile_i & 1) ^ 1, abort_flag);
+                const bool stop = !ok || *abort_flag;
+                if (lane == 0) *stop_flag = stop ? 1 : 0;
+                named_sync(NB_ACC);
+                if (stop) break;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (ok) ok = mbar_wait_warp(bar_full + 8 * s, ph, abort_flag);
+                    named_sync(NB_STAGE0 + s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
             }
         }
     } else {
