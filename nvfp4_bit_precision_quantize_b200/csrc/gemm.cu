@@ -400,16 +400,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     // +128 for B's second 128-row tile, +2 per 64-k step of codes.
                     const int steps = kt < kfull ? 4 : ktail;
                     if (steps == 4) {
+                        if (lane == 0) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                            for (int j = 0; j < 4; ++j) {
+                                tc_cp_scales_if(1u, sf + 4 * j, dsa + 32 * j);
+                                tc_cp_scales_if(1u, sf + 16 + 8 * j, dsb + 32 * j);
+                                tc_cp_scales_if(1u, sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                            }
+                            tc_mma_if(1u, tmem, da, db, sf, sf + 16, acc);
+#pragma unroll
+                            for (int j = 1; j < 4; ++j)
+                                tc_mma_if(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
                         }
-                        tc_mma_if(issue, tmem, da, db, sf, sf + 16, acc);
-#pragma unroll
-                        for (int j = 1; j < 4; ++j)
-                            tc_mma_if(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
+                        __syncwarp();
                     } else {
                         for (int j = 0; j < steps; ++j) {
                             tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);

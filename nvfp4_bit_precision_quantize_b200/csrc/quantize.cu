@@ -10,6 +10,8 @@
 // NVFP4 kontra ograniczenia mikroskalowania" (block 16, E4M3 block scale, FP32
 // tensor scale).  Hadamard transform and stochastic rounding on the Wgrad
 // operands: same page, section "Technologie stabilizujace proces treningowy".
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -147,79 +149,106 @@ __device__ __forceinline__ uint32_t rnd16_of(const uint4 &w, int e) {  // e = id
 
 // ---------------------------------------------------------------------------
 // Pass 2, rowwise: blocks of 16 along the contiguous columns.
-// CTA tile = 128 rows x (32*N) columns; warp w owns rows 16w..16w+15 and each
-// lane one 16-byte chunk of every row (2 (bf16) or 4 (f32) lanes per block).
-// Codes leave as one coalesced 128/64-byte segment per warp and row; the
-// tile's scale atoms are staged in shared memory and written as 16-byte pieces.
+// Persistent CTAs walk 64-row x (32*N)-column tiles in reverse order (the amax
+// pass swept the tensor front to back, so its tail is what L2 still holds);
+// the next tile's loads are in flight while the current tile is encoded.  Warp
+// w owns rows 8w..8w+7 of a tile and each lane one 16-byte chunk of every row
+// (2 (bf16) or 4 (f32) lanes per 16-block).  Codes leave as one coalesced
+// segment per warp and row; a tile fills one half (8 of 16 bytes per atom row)
+// of each of its 128x4 scale atoms, staged in shared memory and written as
+// 8-byte pieces.  Row tiles are counted in pairs so that both halves of every
+// atom are written even when R is not a multiple of 128.
 // ---------------------------------------------------------------------------
 template <typename T, bool SR>
-__global__ void __launch_bounds__(kThreads) quantize_rowwise_kernel(const QParams p) {
+__global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QParams p) {
     constexpr int N = Vec<T>::N;
     constexpr int LPB = 16 / N;          // lanes per 16-block
     constexpr int TILE_C = 32 * N;
+    constexpr int TILE_R = 64;
+    constexpr int RPW = TILE_R / (kThreads / 32);  // rows per warp
     constexpr int ATOMS = TILE_C / 64;   // scale atoms per tile
     __shared__ __align__(16) uint8_t s_sc[ATOMS * 512];
     __shared__ float s_red[kThreads / 32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t rbase = (int64_t)blockIdx.y * 128 + warp * 16;
-    const int64_t c = (int64_t)blockIdx.x * TILE_C + lane * N;
     const T *x = static_cast<const T *>(p.x);
-    const bool col_ok = c < p.C;
-
-    uint4 raw[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int64_t r = rbase + i;
-        raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
-    }
-
-    const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
     const int64_t K = p.C;
     const int64_t KB4 = (K + 63) / 64;
+    const int64_t tiles_c = (p.C + TILE_C - 1) / TILE_C;
+    const int64_t tiles_r = 2 * ((p.R + 127) / 128);
+    const int64_t ntiles = tiles_c * tiles_r;
 
+    auto load = [&](int64_t t, uint4(&buf)[RPW]) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t c = tc * TILE_C + lane * N;
+        const int64_t r0 = tr * TILE_R + warp * RPW;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int64_t r = rbase + i;
-        float v[N];
-        Vec<T>::unpack(raw[i], v);
-        float m = 0.0f;
+        for (int i = 0; i < RPW; ++i) {
+            const int64_t r = r0 + i;
+            buf[i] = (c < p.C && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+
+    int64_t t = ntiles - 1 - (int64_t)blockIdx.x;
+    uint4 cur[RPW], nxt[RPW];
+    if (t >= 0) load(t, cur);
+    const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+
+    for (; t >= 0; t -= gridDim.x) {
+        const int64_t tn = t - gridDim.x;
+        if (tn >= 0) load(tn, nxt);
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t c = tc * TILE_C + lane * N;
+        const bool col_ok = c < p.C;
+        const int half = (int)(tr & 1);  // which 64-row half of the 128-row atoms
 #pragma unroll
-        for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        const BlockScale bs = block_scale(m, s_t);
-        float q[N];
-        if (SR) {
-            const uint64_t idx0 = (uint64_t)r * (uint64_t)K + (uint64_t)c;
-            const uint4 w = sr_words(idx0 & ~7ull, p.seed);
-            const int e0 = (int)(idx0 & 7);
+        for (int i = 0; i < RPW; ++i) {
+            const int rl = warp * RPW + i;  // row within the tile
+            const int64_t r = tr * TILE_R + rl;
+            float v[N];
+            Vec<T>::unpack(cur[i], v);
+            float m = 0.0f;
 #pragma unroll
-            for (int j = 0; j < N; ++j)
-                q[j] = bs.zero ? 0.0f : sr_e2m1_value(__fmul_rn(v[j], bs.inv), rnd16_of(w, e0 + j));
-        } else {
+            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            const BlockScale bs = block_scale(m, s_t);
+            float q[N];
+            if (SR) {
+                const uint64_t idx0 = (uint64_t)r * (uint64_t)K + (uint64_t)c;
+                const uint4 w = sr_words(idx0 & ~7ull, p.seed);
+                const int e0 = (int)(idx0 & 7);
 #pragma unroll
-            for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
+                for (int j = 0; j < N; ++j)
+                    q[j] = bs.zero ? 0.0f : sr_e2m1_value(__fmul_rn(v[j], bs.inv), rnd16_of(w, e0 + j));
+            } else {
+#pragma unroll
+                for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
+            }
+            if (col_ok && r < p.R) {
+                uint8_t *dst = p.codes + r * (K / 2) + c / 2;
+                if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
+                else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+            }
+            if ((lane % LPB) == 0) {
+                const int ra = half * TILE_R + rl, bl = lane / LPB;  // row within the 128-row atom
+                s_sc[(bl >> 2) * 512 + (ra & 31) * 16 + ((ra >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)bs.sb;
+            }
         }
-        if (col_ok && r < p.R) {
-            uint8_t *dst = p.codes + r * (K / 2) + c / 2;
-            if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
-            else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+        __syncthreads();
+        const int64_t atom0 = tc * ATOMS;
+        for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
+            const int atom = i >> 5;
+            if (atom0 + atom < KB4) {
+                const int off = atom * 512 + (i & 31) * 16 + 8 * half;
+                uint8_t *dst = p.scales + ((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half;
+                *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(s_sc + off);
+            }
         }
-        if ((lane % LPB) == 0) {
-            const int rl = warp * 16 + i, bl = lane / LPB;
-            s_sc[(bl >> 2) * 512 + (rl & 31) * 16 + ((rl >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)bs.sb;
-        }
-    }
-    __syncthreads();
-    const int64_t atom0 = (int64_t)blockIdx.x * ATOMS;
-    for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
-        const int atom = i >> 5;
-        if (atom0 + atom < KB4) {
-            uint8_t *dst = p.scales + ((int64_t)blockIdx.y * KB4 + atom0 + atom) * 512 + (i & 31) * 16;
-            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_sc + i * 16);
-        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) cur[i] = nxt[i];
     }
 }
 
@@ -247,8 +276,12 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     __shared__ float s_red[W];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t c = (int64_t)blockIdx.x * TC + lane * N;
-    const int64_t r_warp = (int64_t)blockIdx.y * TR + warp * 32;
+    // Tiles run in reverse order: the amax pass swept the rows front to back, so
+    // the last row tiles are what L2 still holds when this pass starts.
+    const int64_t lin = (int64_t)gridDim.x * gridDim.y - 1 - ((int64_t)blockIdx.y * gridDim.x + blockIdx.x);
+    const int64_t bx = lin % gridDim.x, by = lin / gridDim.x;
+    const int64_t c = bx * TC + lane * N;
+    const int64_t r_warp = by * TR + warp * 32;
     const T *x = static_cast<const T *>(p.x);
     const bool col_ok = c < p.C;
     const int64_t K = p.R;
@@ -316,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     __syncthreads();
 
     // codes: output row (c0 + cl) gets P units of 16 bytes at k-byte offset r0/2 + 16 p
-    const int64_t c0 = (int64_t)blockIdx.x * TC, r0 = (int64_t)blockIdx.y * TR;
+    const int64_t c0 = bx * TC, r0 = by * TR;
     const bool vec16 = (K % 32) == 0;
     for (int i = threadIdx.x; i < TC * P; i += kThreads) {
         const int cl = i / P, pu = i % P;
@@ -338,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     const int64_t rowtiles = (p.C + 127) / 128;
     for (int i = threadIdx.x; i < AR * AC * 32; i += kThreads) {
         const int atom = i >> 5, ar = atom / AC, ac = atom % AC;
-        const int64_t grow = (int64_t)blockIdx.x * AR + ar, gcol = (int64_t)blockIdx.y * AC + ac;
+        const int64_t grow = bx * AR + ar, gcol = by * AC + ac;
         if (grow < rowtiles && gcol < KB4) {
             uint8_t *dst = p.scales + (grow * KB4 + gcol) * 512 + (i & 31) * 16;
             *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_sc + i * 16);
@@ -376,7 +409,8 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
               a.tensor_scale};
     constexpr int N = Vec<T>::N;
     if (!a.colwise) {
-        dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 127) / 128));
+        const int64_t tiles = ((a.C + 32 * N - 1) / (32 * N)) * 2 * ((a.R + 127) / 128);
+        const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
         if (a.sr) quantize_rowwise_kernel<T, true><<<grid, kThreads, 0, s>>>(p);
         else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);
     } else {
