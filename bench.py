@@ -2,8 +2,9 @@
 Mamba-Transformer layer shape on B200, through the C ABI.
 
 A step = up-projection Fprop, squared ReLU, down-projection Fprop, then both
-layers' Dgrad and Wgrad (RHT + SR on the Wgrad operands): 12 two-pass NVFP4
-quantisations, 6 block-scaled NVFP4 GEMMs, 2 elementwise kernels.  With N > 1
+layers' Dgrad and Wgrad (RHT + SR on the Wgrad operands): 12 NVFP4 operands
+from two-pass quantisations (each weight's two operands from one read), 6
+block-scaled NVFP4 GEMMs, 2 elementwise kernels.  With N > 1
 GPUs (torchrun) every rank runs the step on its own token shard and the weight
 gradients are summed over NCCL (weak scaling).
 
@@ -38,7 +39,10 @@ SEED = 1234
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 FP4_PER_BF16 = 4.0                                 # nominal dense ratio 9 / 2.25 PFLOP/s
 WORKLOAD = ("mlp_fwd_bwd: tokens 8192, hidden 5120, ffn 20480, up -> relu^2 -> down; "
-            "6 NVFP4 GEMMs + 12 NVFP4 quantisations (RHT+SR on Wgrad operands) + 2 relu^2 kernels")
+            "6 NVFP4 GEMMs + 12 NVFP4 operands (8 single quantisations, 2 dual-orientation ones for the "
+            "weights; RHT+SR on Wgrad operands) + 2 relu^2 kernels")
+QUANT_BYTES_SINGLE = 4.5625   # bf16, two passes: read 2 + 2, write 0.5 + 1/16 bytes per element
+QUANT_BYTES_DUAL = 5.125      # bf16, two passes, two outputs: read 2 + 2, write 2 x (0.5 + 1/16)
 
 
 def peaks():
@@ -124,7 +128,7 @@ class MlpStep:
         self.dW2 = torch.empty((HID, FFN), dtype=torch.float32, device=device)
         self.ws = B.workspace(max(B.nvfp4_linear_workspace_size(M_TOK, FFN, HID),
                                   B.nvfp4_linear_workspace_size(M_TOK, HID, FFN)), device)
-        self.qws = B.workspace(B.nvfp4_quantize_workspace_size(), device)
+        self.qws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), device)
         mk = B.empty_nvfp4
         # NVFP4 operands of the explicit call sequence (same work as linear_fwd/bwd)
         self.q = {
@@ -145,7 +149,17 @@ class MlpStep:
                          ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
-            ev.append(("quant", x.numel(), torch.cuda.Event(enable_timing=True)))
+            ev.append(("quant", x.numel() * QUANT_BYTES_SINGLE, torch.cuda.Event(enable_timing=True)))
+            ev[-1][2].record()
+
+    def _dual(self, x, key_r, key_c, sr=False, rht=False, ev=None):
+        """Rowwise RTN and colwise operands of one tensor from one read."""
+        B = self.B
+        B.nvfp4_quantize_dual(x, col_rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, col_rht=rht, seed=SEED,
+                              out_row=self.q[key_r], out_col=self.q[key_c], ws=self.qws)
+        self.launches += B.nvfp4_last_launch_count()
+        if ev is not None:
+            ev.append(("quant", x.numel() * QUANT_BYTES_DUAL, torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
 
     def _gemm(self, a, b, out, ev=None):
@@ -163,9 +177,11 @@ class MlpStep:
         if ev is not None:
             ev.append(("start", 0, torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
-        # forward
+        # forward.  A weight's two operands (rowwise, colwise without RHT) come from one
+        # dual-orientation call; where the colwise operand carries the Hadamard transform
+        # (and SR) that pass is ALU-bound and the two single calls are faster.
         self._quant(d["X"], "X_r", ev=ev)
-        self._quant(d["W1"], "W1_r", ev=ev)
+        self._dual(d["W1"], "W1_r", "W1_c", ev=ev)
         self._gemm("X_r", "W1_r", self.Y1, ev)
         B.nvfp4_relu2_fwd(self.Y1, out=self.h)
         self.launches += B.nvfp4_last_launch_count()
@@ -173,11 +189,10 @@ class MlpStep:
             ev.append(("relu2", self.Y1.numel(), torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
         self._quant(self.h, "h_r", ev=ev)
-        self._quant(d["W2"], "W2_r", ev=ev)
+        self._dual(d["W2"], "W2_r", "W2_c", ev=ev)
         self._gemm("h_r", "W2_r", self.Y2, ev)
         # down-projection backward: dh = dY2 . W2, dW2 = dY2^T h
         self._quant(d["dY2"], "dY2_r", ev=ev)
-        self._quant(d["W2"], "W2_c", colwise=True, ev=ev)
         self._gemm("dY2_r", "W2_c", self.dh, ev)
         self._quant(d["dY2"], "dY2_c", colwise=True, sr=True, rht=True, ev=ev)
         self._quant(self.h, "h_c", colwise=True, rht=True, ev=ev)
@@ -189,7 +204,6 @@ class MlpStep:
             ev[-1][2].record()
         # up-projection backward: dX = dY1 . W1, dW1 = dY1^T X
         self._quant(self.dY1, "dY1_r", ev=ev)
-        self._quant(d["W1"], "W1_c", colwise=True, ev=ev)
         self._gemm("dY1_r", "W1_c", self.dX, ev)
         self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, ev=ev)
         self._quant(d["X"], "X_c", colwise=True, rht=True, ev=ev)
@@ -385,9 +399,8 @@ def run_ours(args):
         gemm_flops = g[1] / g[2]
         gemm_tflops = gemm_flops / (gemm_ms / 1e3) / 1e12
         fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
-        # two-pass quantise of bf16: read 2 + 2 bytes, write 0.5 + 1/16 bytes per element
-        q_bytes = q[1] * 4.5625
-        q_gbs = q_bytes / (q[0] / 1e3) / 1e9
+        # algorithmic bytes of the quantise calls (two-pass, dual-orientation: 5.125 B per element)
+        q_gbs = q[1] / (q[0] / 1e3) / 1e9
         tr = traffic_record("gemm_nvfp4_kernel")
         line = {
             "metric": METRIC, "value": nproc * GEMM_FLOPS / (ms_max / 1e3) / 1e12, "unit": "TFLOP/s",
@@ -405,8 +418,10 @@ def run_ours(args):
                          "peak_source": "%s bf16_tflops_sustained x %.0f (nominal dense fp4/bf16)" % (src,
                                                                                             FP4_PER_BF16),
                          "launch_ms": gemm_ms, "flop_per_launch": gemm_flops},
-            "roofline_quantize": {"bound": "hbm", "achieved": q_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                  "frac": q_gbs / pk["hbm_gbs"], "bytes_per_elem": 4.5625,
+            "roofline_quantize": {"bound": "hbm", "kernels": "amax*, quantize_rowwise, quantize_colwise (+dual)",
+                                  "achieved": q_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": q_gbs / pk["hbm_gbs"],
+                                  "bytes_per_elem": {"single": QUANT_BYTES_SINGLE, "dual": QUANT_BYTES_DUAL},
                                   "calls_per_step": q[2] // args.steps, "peak_source": src + " hbm_gbs",
                                   "call_ms": q[0] / q[2]},
             "breakdown_ms_per_step": {k: v[0] / args.steps for k, v in stats.items()},
@@ -457,6 +472,13 @@ def run_profile_case(case):
         q = None
         for _ in range(3):
             q = B.nvfp4_quantize(x, out=q, ws=ws, seed=SEED, **kw)
+    elif case == "quant_dual":  # the step's dY1: rowwise RTN + colwise RHT + SR from one read
+        x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, FFN), 1e-3))).to(dev)
+        ws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), dev)
+        r = c = None
+        for _ in range(3):
+            r, c = B.nvfp4_quantize_dual(x, col_rounding=B.NVFP4_SR, col_rht=True, seed=SEED, out_row=r, out_col=c,
+                                         ws=ws)
     else:
         raise SystemExit("unknown profile case " + case)
     torch.cuda.synchronize()
@@ -470,7 +492,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy"],
+    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy", "quant_dual"],
                     help="run one kernel a few times for an ncu capture instead of the benchmark")
     args = ap.parse_args()
     if args.profile_case:

@@ -116,6 +116,30 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t 
                             const float *amax_in, const nvfp4_tensor *out,
                             void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* Both NVFP4 operands of one tensor from one read of it (the layer's
+ * backward pass needs dY rowwise for Dgrad and colwise with the Hadamard
+ * transform and stochastic rounding for Wgrad; the same holds for every
+ * tensor the MLP step quantises in both orientations).  The results are
+ * bit-identical to
+ *   nvfp4_quantize(x, ..., NVFP4_ROWWISE, NVFP4_RTN, 0, seed, amax_row_in, out_row, ...)
+ *   nvfp4_quantize(x, ..., NVFP4_COLWISE, col_rounding, col_rht, seed, amax_col_in, out_col, ...)
+ * (format: aisight.pl, section "Architektura NVFP4 kontra ograniczenia
+ * mikroskalowania"; Hadamard transform and stochastic rounding on the Wgrad
+ * operands: same page, section "Technologie stabilizujace proces
+ * treningowy").  x, R, C, ld, dtype, out_row ([R x C]) and out_col ([C x R])
+ * follow nvfp4_quantize for their orientation, so both sets of shape and
+ * alignment rules apply.  workspace: >= nvfp4_quantize_dual_workspace_size()
+ * bytes, 16-byte aligned, zeroed status word, unless both amax_*_in are given.
+ * Passes: one amax pass computing max|x| and, with col_rht, max|RHT(x)| in the
+ * same read (skipped when both amax values are supplied), then one quantise
+ * pass writing both outputs.  Errors as nvfp4_quantize. */
+NVFP4_API size_t nvfp4_quantize_dual_workspace_size(void);
+NVFP4_API nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
+                                           int col_rounding, int col_rht, uint64_t seed,
+                                           const float *amax_row_in, const float *amax_col_in,
+                                           const nvfp4_tensor *out_row, const nvfp4_tensor *out_col,
+                                           void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /*
  * nvfp4_gemm -- C[M x N] = (A . B^T) * sA * sB with A = [M x K], B = [N x K]
  * NVFP4 tensors (the block-scaled GEMM used for Fprop, Dgrad and Wgrad; 4-bit
@@ -152,7 +176,8 @@ NVFP4_API nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, i
  * The random Hadamard transform and stochastic rounding apply to the Wgrad
  * operands only (aisight.pl, section "Technologie stabilizujace proces
  * treningowy"); both Wgrad operands use the same signs, from `seed`, which
- * also keys the SR draws.  Requires M % 64 == 0, N % 64 == 0, K % 64 == 0.
+ * also keys the SR draws.  dY's two operands come from one read of dY
+ * (nvfp4_quantize_dual).  Requires M % 64 == 0, N % 64 == 0, K % 64 == 0.
  */
 NVFP4_API nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void *dX, float *dW,
                               int64_t M, int64_t N, int64_t K, nvfp4_dtype dtype,
@@ -197,6 +222,17 @@ NVFP4_API nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, 
  * word: NVFP4_OK, NVFP4_ERR_DEVICE_TIMEOUT, or NVFP4_ERR_CUDA if the stream
  * reports an error. */
 NVFP4_API nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream);
+
+/* Self-test of the device-timeout path (no counterpart on the pages): one
+ * thread waits on an mbarrier that nothing arrives on, with the same bounded
+ * loop the GEMM uses but a limit of limit_ns nanoseconds (1 .. 2e9), then
+ * records NVFP4_ERR_DEVICE_TIMEOUT in the workspace status word (workspace:
+ * >= 256 bytes, 16-byte aligned, device memory, caller-owned) and returns.
+ * Asynchronous; the following nvfp4_check() reports (and clears) the status.
+ * Launch errors: NVFP4_ERR_WORKSPACE, NVFP4_ERR_ALIGNMENT,
+ * NVFP4_ERR_INVALID_ARG (limit out of range), NVFP4_ERR_UNSUPPORTED_DEVICE. */
+NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_bytes, uint64_t limit_ns,
+                                                   cudaStream_t stream);
 
 /* Number of kernel launches the most recent successful call on this host
  * thread issued (launch accounting for benchmarks). */

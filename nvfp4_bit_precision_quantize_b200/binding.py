@@ -33,7 +33,8 @@ NVFP4_SR = 1
 EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_size", "nvfp4_quantize",
            "nvfp4_gemm", "nvfp4_linear_workspace_size", "nvfp4_linear_fwd", "nvfp4_linear_bwd",
            "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
-           "nvfp4_status_string", "nvfp4_linear_fwd_noalloc")
+           "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
+           "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual")
 
 
 class CTensor(C.Structure):
@@ -75,6 +76,9 @@ def load():
         "nvfp4_last_launch_count": (i32, []),
         "nvfp4_status_string": (C.c_char_p, [i32]),
         "nvfp4_linear_fwd_noalloc": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp]),
+        "nvfp4_selftest_wait_timeout": (i32, [vp, sz, u64, vp]),
+        "nvfp4_quantize_dual_workspace_size": (sz, []),
+        "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -169,6 +173,25 @@ def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, 
     return out
 
 
+def nvfp4_quantize_dual_workspace_size():
+    return load().nvfp4_quantize_dual_workspace_size()
+
+
+def nvfp4_quantize_dual(x, col_rounding=NVFP4_RTN, col_rht=False, seed=1234, amax_row_in=None, amax_col_in=None,
+                        out_row=None, out_col=None, ws=None, stream=None):
+    """Rowwise (RTN) and colwise NVFP4 of one 2-D tensor from one read; returns (row, col)."""
+    R, Cc = x.shape
+    out_row = out_row or empty_nvfp4(R, Cc, x.device)
+    out_col = out_col or empty_nvfp4(Cc, R, x.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), x.device)
+    cr, cc = out_row.c(), out_col.c()
+    st = load().nvfp4_quantize_dual(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), col_rounding,
+                                    int(bool(col_rht)), seed, _ptr(amax_row_in), _ptr(amax_col_in), C.byref(cr),
+                                    C.byref(cc), _ptr(ws), ws.numel(), _stream(stream))
+    _ok(st, "nvfp4_quantize_dual")
+    return out_row, out_col
+
+
 def nvfp4_gemm(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
     """C = (A . B^T) * sA * sB for NVFP4 tensors A [M x K], B [N x K]."""
     M, N = A.rows, B.rows
@@ -232,6 +255,12 @@ def nvfp4_relu2_bwd(dh, y, out=None, stream=None):
 def nvfp4_check(ws, stream=None):
     """Synchronise and read/clear the workspace status word; raises on a device error."""
     _ok(load().nvfp4_check(_ptr(ws), _stream(stream)), "nvfp4_check")
+
+
+def nvfp4_selftest_wait_timeout(ws, limit_ns, stream=None):
+    """Launch the device-timeout self-test (its status is read by nvfp4_check)."""
+    _ok(load().nvfp4_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(limit_ns), _stream(stream)),
+        "nvfp4_selftest_wait_timeout")
 
 
 def nvfp4_last_launch_count():

@@ -122,8 +122,8 @@ struct Carver {
         return t;
     }
 };
-constexpr size_t kScalarsOff = kQuantizeWorkspace;            // 4 tensor scales
-constexpr size_t kBuffersOff = kQuantizeWorkspace + 256;
+constexpr size_t kScalarsOff = kDualWorkspace;                // 4 tensor scales (after two amax partial sets)
+constexpr size_t kBuffersOff = kDualWorkspace + 256;
 
 size_t fwd_bytes(int64_t M, int64_t N, int64_t K) {
     Carver c{nullptr, kBuffersOff};
@@ -188,6 +188,32 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nv
     return from_cuda(launch_gemm(g, stream, launches));
 }
 
+nvfp4_status dual_impl(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int col_rounding,
+                       int col_rht, uint64_t seed, const float *amax_row_in, const float *amax_col_in,
+                       const nvfp4_tensor *out_row, const nvfp4_tensor *out_col, void *ws, cudaStream_t stream,
+                       int *launches) {
+    DualQuantizeArgs a;
+    a.x = x;
+    a.bf16 = dtype == NVFP4_DTYPE_BF16;
+    a.R = R;
+    a.C = C;
+    a.ld = ld;
+    a.col_sr = col_rounding == NVFP4_SR;
+    a.col_rht = col_rht != 0;
+    a.seed = seed;
+    a.amax_row_in = amax_row_in;
+    a.amax_col_in = amax_col_in;
+    a.row_codes = out_row->codes;
+    a.row_scales = out_row->scales;
+    a.row_tensor_scale = out_row->tensor_scale;
+    a.col_codes = out_col->codes;
+    a.col_scales = out_col->scales;
+    a.col_tensor_scale = out_col->tensor_scale;
+    a.row_partials = ws ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kStatusBytes) : nullptr;
+    a.col_partials = a.row_partials ? a.row_partials + kMaxPartials : nullptr;
+    return from_cuda(launch_quantize_dual(a, stream, launches));
+}
+
 }  // namespace
 
 extern "C" {
@@ -222,6 +248,28 @@ nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t R, int64_t
     st = quantize_impl(x, dtype, R, C, ld, orientation, rounding, rht, seed, amax_in, out, workspace, stream,
                        &call.launches);
     return call.done(st);
+}
+
+size_t nvfp4_quantize_dual_workspace_size(void) { return kDualWorkspace; }
+
+nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
+                                 int col_rounding, int col_rht, uint64_t seed, const float *amax_row_in,
+                                 const float *amax_col_in, const nvfp4_tensor *out_row,
+                                 const nvfp4_tensor *out_col, void *workspace, size_t ws_bytes,
+                                 cudaStream_t stream) {
+    Call call;
+    // each orientation's own checks; the dual workspace holds both amax partial sets
+    nvfp4_status st = validate_quantize(x, dtype, R, C, ld, NVFP4_ROWWISE, NVFP4_RTN, 0, amax_row_in, out_row,
+                                        workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    st = validate_quantize(x, dtype, R, C, ld, NVFP4_COLWISE, col_rounding, col_rht, amax_col_in, out_col,
+                           workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    if (R > 0 && C > 0 && !(amax_row_in && amax_col_in) && (!workspace || ws_bytes < kDualWorkspace))
+        return NVFP4_ERR_WORKSPACE;
+    if ((st = check_device()) != NVFP4_OK) return st;
+    return call.done(dual_impl(x, dtype, R, C, ld, col_rounding, col_rht, seed, amax_row_in, amax_col_in, out_row,
+                               out_col, workspace, stream, &call.launches));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype, int64_t ldc,
@@ -289,17 +337,17 @@ nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void
         (st = validate_gemm(&dy_c, &x_c, dW, NVFP4_DTYPE_F32, K, ws, ws_bytes)))
         return st;
     if ((st = check_device()) != NVFP4_OK) return st;
+    // dY's two operands (Dgrad rowwise, Wgrad colwise with RHT + SR) from one read
+    if ((st = dual_impl(dY, dtype, M, N, N, NVFP4_SR, 1, seed, nullptr, nullptr, &dy_r, &dy_c, ws, stream,
+                        &call.launches)))
+        return st;
     // Dgrad: dX = dY . W
-    if ((st = quantize_impl(dY, dtype, M, N, N, NVFP4_ROWWISE, NVFP4_RTN, 0, seed, nullptr, &dy_r, ws, stream,
-                            &call.launches)) ||
-        (st = quantize_impl(W, dtype, N, K, K, NVFP4_COLWISE, NVFP4_RTN, 0, seed, nullptr, &w_c, ws, stream,
+    if ((st = quantize_impl(W, dtype, N, K, K, NVFP4_COLWISE, NVFP4_RTN, 0, seed, nullptr, &w_c, ws, stream,
                             &call.launches)) ||
         (st = gemm_impl(&dy_r, &w_c, dX, dx_dtype, K, ws, stream, &call.launches)))
         return st;
     // Wgrad: dW = dY^T . X with the Hadamard transform on both operands, SR on dY
-    if ((st = quantize_impl(dY, dtype, M, N, N, NVFP4_COLWISE, NVFP4_SR, 1, seed, nullptr, &dy_c, ws, stream,
-                            &call.launches)) ||
-        (st = quantize_impl(X, dtype, M, K, K, NVFP4_COLWISE, NVFP4_RTN, 1, seed, nullptr, &x_c, ws, stream,
+    if ((st = quantize_impl(X, dtype, M, K, K, NVFP4_COLWISE, NVFP4_RTN, 1, seed, nullptr, &x_c, ws, stream,
                             &call.launches)) ||
         (st = gemm_impl(&dy_c, &x_c, dW, NVFP4_DTYPE_F32, K, ws, stream, &call.launches)))
         return st;
@@ -338,6 +386,16 @@ nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream) {
         return status == NVFP4_ERR_DEVICE_TIMEOUT ? NVFP4_ERR_DEVICE_TIMEOUT : NVFP4_ERR_CUDA;
     }
     return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_bytes, uint64_t limit_ns, cudaStream_t stream) {
+    Call call;
+    if (!workspace || ws_bytes < kStatusBytes) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    if (limit_ns == 0 || limit_ns > 2000000000ull) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    return call.done(from_cuda(launch_wait_timeout(static_cast<int *>(workspace), limit_ns, stream, &call.launches)));
 }
 
 int nvfp4_last_launch_count(void) { return g_last_launches; }

@@ -9,6 +9,7 @@ namespace nvfp4 {
 constexpr int kMaxPartials = 1024;          // per-CTA amax partials in a quantize workspace
 constexpr size_t kStatusBytes = 256;        // status word region at the start of a workspace
 constexpr size_t kQuantizeWorkspace = kStatusBytes + kMaxPartials * sizeof(float);
+constexpr size_t kDualWorkspace = kStatusBytes + 2 * kMaxPartials * sizeof(float);
 
 struct QuantizeArgs {
     const void *x;
@@ -21,6 +22,21 @@ struct QuantizeArgs {
     uint8_t *scales;
     float *tensor_scale;
     float *partials;        // kMaxPartials floats (unused when amax_in is set)
+};
+
+// Rowwise RTN and colwise (RTN/SR, optional RHT) outputs of one tensor from one read.
+struct DualQuantizeArgs {
+    const void *x;
+    bool bf16;
+    int64_t R, C, ld;
+    bool col_sr, col_rht;
+    uint64_t seed;
+    const float *amax_row_in, *amax_col_in;  // optional
+    uint8_t *row_codes, *row_scales;
+    float *row_tensor_scale;
+    uint8_t *col_codes, *col_scales;
+    float *col_tensor_scale;
+    float *row_partials, *col_partials;      // kMaxPartials floats each
 };
 
 struct GemmArgs {
@@ -37,10 +53,14 @@ struct GemmArgs {
 
 // Each launcher adds the number of kernels it launched to *launches.
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t s, int *launches);
 cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t s,
                              int *launches);
+
+// One bounded wait on an mbarrier nothing arrives on; records the timeout status.
+cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);
 
 int num_sms();  // SM count of the current device (cached)
 

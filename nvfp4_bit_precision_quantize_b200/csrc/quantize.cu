@@ -120,6 +120,64 @@ __global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict_
     }
 }
 
+// ---------------------------------------------------------------------------
+// Pass 1c: both max |x| and max |RHT(x)| (transform down 16-row groups of every
+// column) from one read, for the dual quantiser; units as in pass 1b.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) amax_dual_kernel(const T *__restrict__ x, int64_t R, int64_t C,
+                                                             int64_t ld, uint64_t seed,
+                                                             float *__restrict__ partials_plain,
+                                                             float *__restrict__ partials_rht) {
+    constexpr int N = Vec<T>::N;
+    __shared__ float s_red[2][kThreads / 32];
+    const uint32_t signs = rht_sign_bits(seed);
+    const int64_t chunks = C / N;
+    const int64_t total = (R / 16) * chunks;
+    float m0 = 0.0f, m1 = 0.0f;
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * kThreads) {
+        const int64_t g = u / chunks, cc = u - g * chunks;
+        const T *p = x + (g * 16) * ld + cc * N;
+        uint4 raw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float t[N];
+                Vec<T>::unpack(raw[i], t);
+                v[i] = t[j];
+                m0 = fmaxf(m0, fabsf(v[i]));
+            }
+            rht16(v, signs);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m1 = fmaxf(m1, fabsf(v[i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        s_red[0][threadIdx.x >> 5] = m0;
+        s_red[1][threadIdx.x >> 5] = m1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b0 = 0.0f, b1 = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            b0 = fmaxf(b0, s_red[0][w]);
+            b1 = fmaxf(b1, s_red[1][w]);
+        }
+        partials_plain[blockIdx.x] = b0;
+        partials_rht[blockIdx.x] = b1;
+    }
+}
+
 struct QParams {
     const void *x;
     int64_t R, C, ld;
@@ -130,6 +188,12 @@ struct QParams {
     uint8_t *codes;
     uint8_t *scales;
     float *tensor_scale;
+    // dual quantiser only: the rowwise (RTN) output of the same tensor
+    const float *row_amax_in;
+    const float *row_partials;
+    uint8_t *row_codes;
+    uint8_t *row_scales;
+    float *row_tensor_scale;
 };
 
 __device__ __forceinline__ float tensor_amax(const QParams &p, float *s_red) {
@@ -262,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
 // an xor swizzle so both the scatter and the row-contiguous read-out are free
 // of bank conflicts beyond the 4-wavefront minimum.
 // ---------------------------------------------------------------------------
-template <typename T, bool SR, bool RHT>
+template <typename T, bool SR, bool RHT, bool DUAL>
 __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QParams p) {
     constexpr int N = Vec<T>::N;
     constexpr int W = kThreads / 32;     // warps
@@ -274,6 +338,10 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     __shared__ __align__(16) uint4 s_units[N * P * 32];
     __shared__ __align__(16) uint8_t s_sc[AR * AC * 512];
     __shared__ float s_red[W];
+    constexpr int LPB = 16 / N;          // dual: lanes per rowwise 16-block
+    constexpr int ARR = TR / 128;        // dual: rowwise scale-atom rows per tile
+    constexpr int ACR = TC / 64;         // dual: rowwise scale-atom columns per tile
+    __shared__ __align__(16) uint8_t s_scr[DUAL ? ARR * ACR * 512 : 16];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // Tiles run in reverse order: the amax pass swept the rows front to back, so
@@ -295,10 +363,16 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
         raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
     }
     const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+    float s_t_row = 0.0f;
+    if (DUAL)
+        s_t_row = tensor_scale_from_amax(p.row_amax_in ? *p.row_amax_in
+                                                       : reduce_partials_max(p.row_partials, p.num_partials, s_red));
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        *p.tensor_scale = s_t;
+        if (DUAL) *p.row_tensor_scale = s_t_row;
+    }
     const uint32_t signs = RHT ? rht_sign_bits(p.seed) : 0u;
 
-    uint2 cw[N][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int64_t rg = r_warp + 16 * h;
@@ -307,6 +381,35 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
             for (int i = 0; i < 16; ++i) {
                 const int64_t r = rg + i;
                 raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        if (DUAL) {
+            // Rowwise RTN encode of the same 16 rows: a lane holds N of a row's 16-block,
+            // the partner lane(s) the rest (as in the rowwise quantiser).
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int64_t r = rg + i;
+                float v[N];
+                Vec<T>::unpack(raw[i], v);
+                float m = 0.0f;
+#pragma unroll
+                for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                const BlockScale bs = block_scale(m, s_t_row);
+                float q[N];
+#pragma unroll
+                for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
+                if (col_ok && r < p.R) {
+                    uint8_t *dst = p.row_codes + r * (p.C / 2) + c / 2;
+                    if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
+                    else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+                }
+                if ((lane % LPB) == 0) {
+                    const int rl = warp * 32 + 16 * h + i, bl = lane / LPB;
+                    s_scr[((rl >> 7) * ACR + (bl >> 2)) * 512 + (rl & 31) * 16 + ((rl >> 5) & 3) * 4 + (bl & 3)] =
+                        (uint8_t)bs.sb;
+                }
             }
         }
 #pragma unroll
@@ -335,16 +438,15 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
 #pragma unroll
                 for (int i = 0; i < 16; ++i) q[i] = bs.zero ? 0.0f : __fmul_rn(v[i], bs.inv);
             }
-            cw[j][h] = make_uint2(e2m1x8(q), e2m1x8(q + 8));
+            {  // this group's 8 code bytes: half h of the lane's 16-byte unit for column j
+                const int qu = j * P + warp;
+                reinterpret_cast<uint2 *>(s_units)[(qu * 32 + (lane ^ (qu & 7))) * 2 + h] =
+                    make_uint2(e2m1x8(q), e2m1x8(q + 8));
+            }
             const int cl = lane * N + j, gl = warp * 2 + h;
             s_sc[((cl >> 7) * AC + (gl >> 2)) * 512 + (cl & 31) * 16 + ((cl >> 5) & 3) * 4 + (gl & 3)] =
                 (uint8_t)bs.sb;
         }
-    }
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-        const int q = j * P + warp;
-        s_units[q * 32 + (lane ^ (q & 7))] = make_uint4(cw[j][0].x, cw[j][0].y, cw[j][1].x, cw[j][1].y);
     }
     __syncthreads();
 
@@ -364,6 +466,17 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
             } else {  // rows only 8-byte aligned (K % 32 == 16), or the K tail
                 *reinterpret_cast<uint2 *>(dst) = make_uint2(u.x, u.y);
                 if (rem >= 32) *reinterpret_cast<uint2 *>(dst + 8) = make_uint2(u.z, u.w);
+            }
+        }
+    }
+    if (DUAL) {  // rowwise scale atoms of the tile: ARR x ACR
+        const int64_t rowtiles_r = (p.R + 127) / 128, kb4_r = (p.C + 63) / 64;
+        for (int i = threadIdx.x; i < ARR * ACR * 32; i += kThreads) {
+            const int atom = i >> 5, ar = atom / ACR, ac = atom % ACR;
+            const int64_t grow = by * ARR + ar, gcol = bx * ACR + ac;
+            if (grow < rowtiles_r && gcol < kb4_r) {
+                uint8_t *dst = p.row_scales + (grow * kb4_r + gcol) * 512 + (i & 31) * 16;
+                *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_scr + i * 16);
             }
         }
     }
@@ -415,16 +528,61 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
         else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);
     } else {
         dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 255) / 256));
-        if (a.sr && a.rht) quantize_colwise_kernel<T, true, true><<<grid, kThreads, 0, s>>>(p);
-        else if (a.sr) quantize_colwise_kernel<T, true, false><<<grid, kThreads, 0, s>>>(p);
-        else if (a.rht) quantize_colwise_kernel<T, false, true><<<grid, kThreads, 0, s>>>(p);
-        else quantize_colwise_kernel<T, false, false><<<grid, kThreads, 0, s>>>(p);
+        if (a.sr && a.rht) quantize_colwise_kernel<T, true, true, false><<<grid, kThreads, 0, s>>>(p);
+        else if (a.sr) quantize_colwise_kernel<T, true, false, false><<<grid, kThreads, 0, s>>>(p);
+        else if (a.rht) quantize_colwise_kernel<T, false, true, false><<<grid, kThreads, 0, s>>>(p);
+        else quantize_colwise_kernel<T, false, false, false><<<grid, kThreads, 0, s>>>(p);
     }
     ++*launches;
     return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t run_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches) {
+    const T *x = static_cast<const T *>(a.x);
+    constexpr int N = Vec<T>::N;
+    int num_partials = 0;
+    const float *col_partials = a.col_rht ? a.col_partials : a.row_partials;  // no RHT: one amax serves both
+    if (!(a.amax_row_in && a.amax_col_in)) {
+        const int sms = num_sms();
+        if (a.col_rht) {
+            const int64_t units = (a.R / 16) * (a.C / N);
+            num_partials = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                                  std::max<int64_t>(1, (units + kThreads - 1) / kThreads));
+            amax_dual_kernel<T><<<num_partials, kThreads, 0, s>>>(x, a.R, a.C, a.ld, a.seed, a.row_partials,
+                                                                  a.col_partials);
+        } else {
+            const int64_t chunks = a.R * (a.C / N);
+            num_partials = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                                  std::max<int64_t>(1, (chunks + kThreads - 1) / kThreads));
+            amax_kernel<T><<<num_partials, kThreads, 0, s>>>(x, a.R, a.C, a.ld, a.row_partials);
+        }
+        ++*launches;
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    QParams p{a.x, a.R, a.C, a.ld, a.seed, a.amax_col_in, col_partials, num_partials, a.col_codes, a.col_scales,
+              a.col_tensor_scale, a.amax_row_in, a.row_partials, a.row_codes, a.row_scales, a.row_tensor_scale};
+    dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 255) / 256));
+    if (a.col_sr && a.col_rht) quantize_colwise_kernel<T, true, true, true><<<grid, kThreads, 0, s>>>(p);
+    else if (a.col_sr) quantize_colwise_kernel<T, true, false, true><<<grid, kThreads, 0, s>>>(p);
+    else if (a.col_rht) quantize_colwise_kernel<T, false, true, true><<<grid, kThreads, 0, s>>>(p);
+    else quantize_colwise_kernel<T, false, false, true><<<grid, kThreads, 0, s>>>(p);
+    ++*launches;
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches) {
+    if (a.R == 0 || a.C == 0) {
+        tensor_scale_only_kernel<<<1, 1, 0, s>>>(a.amax_row_in, a.row_tensor_scale);
+        tensor_scale_only_kernel<<<1, 1, 0, s>>>(a.amax_col_in, a.col_tensor_scale);
+        *launches += 2;
+        return cudaGetLastError();
+    }
+    return a.bf16 ? run_dual<uint16_t>(a, s, launches) : run_dual<float>(a, s, launches);
+}
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches) {
     if (a.R == 0 || a.C == 0) {

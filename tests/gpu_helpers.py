@@ -35,6 +35,11 @@ def first_mismatch(a, b):
 def check_quantize(x, colwise=False, sr=False, rht=False, seed=1234, amax_in=None):
     """Bit-exact comparison of codes, scales (and their zero padding) and tensor scale."""
     q = gpu_quantize(x, colwise, sr, rht, seed, amax_in)
+    return compare_quantize(q, x, colwise, sr, rht, seed, amax_in)
+
+
+def compare_quantize(q, x, colwise=False, sr=False, rht=False, seed=1234, amax_in=None):
+    """Bit-exact comparison of a GPU NVFP4 tensor q with the oracle's quantisation of x."""
     oc, osc, ots, _ = oracle.quantize(x, colwise=colwise, sr=sr, rht=rht, seed=seed, amax_in=amax_in)
     rows, k = oc.shape[0], oc.shape[1] * 2
     gts = q.tensor_scale.cpu().numpy()[0]

@@ -113,3 +113,32 @@ def test_linear_rejections(lib):
                                 1, p(0x6000), ws, None) == E.NVFP4_ERR_SHAPE
     assert lib.nvfp4_relu2_fwd(p(0x1001), p(0x2000), 16, None) == E.NVFP4_ERR_ALIGNMENT
     assert lib.nvfp4_relu2_bwd(None, p(0x2000), p(0x3000), 16, None) == E.NVFP4_ERR_INVALID_ARG
+
+
+def test_selftest_rejections(lib):
+    ws = C.c_void_p(0x20000)
+    assert lib.nvfp4_selftest_wait_timeout(None, 256, 1000, None) == binding.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_selftest_wait_timeout(ws, 255, 1000, None) == binding.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_selftest_wait_timeout(C.c_void_p(0x20008), 256, 1000, None) == binding.NVFP4_ERR_ALIGNMENT
+    assert lib.nvfp4_selftest_wait_timeout(ws, 256, 0, None) == binding.NVFP4_ERR_INVALID_ARG
+    assert lib.nvfp4_selftest_wait_timeout(ws, 256, 3_000_000_000, None) == binding.NVFP4_ERR_INVALID_ARG
+
+
+def test_quantize_dual_rejections(lib):
+    ws = C.c_void_p(0x20000)
+    row, col = _tensor(64, 64), _tensor(64, 64)
+
+    def dual(x=0x10000, dtype=1, R=64, Cc=64, ld=64, rnd=0, rht=0, r=None, c=None, w=ws, wsb=1 << 20, ar=None,
+             ac=None):
+        return lib.nvfp4_quantize_dual(C.c_void_p(x), dtype, R, Cc, ld, rnd, rht, 7, ar, ac,
+                                       C.byref(r if r is not None else row), C.byref(c if c is not None else col),
+                                       w, wsb, None)
+    assert lib.nvfp4_quantize_dual_workspace_size() >= 256 + 2 * 4 * 1024
+    assert dual(rnd=2) == binding.NVFP4_ERR_INVALID_ARG
+    assert dual(rht=2) == binding.NVFP4_ERR_INVALID_ARG
+    assert dual(R=60, r=_tensor(60, 64), c=_tensor(64, 60)) == binding.NVFP4_ERR_SHAPE        # colwise needs R % 16
+    assert dual(Cc=72, ld=72, r=_tensor(64, 72), c=_tensor(72, 64)) == binding.NVFP4_ERR_SHAPE  # rowwise needs C % 16
+    assert dual(c=_tensor(32, 64)) == binding.NVFP4_ERR_SHAPE
+    assert dual(wsb=4352) == binding.NVFP4_ERR_WORKSPACE              # single-orientation size is not enough
+    assert dual(w=None) == binding.NVFP4_ERR_WORKSPACE
+    assert dual(x=0x10008) == binding.NVFP4_ERR_ALIGNMENT
