@@ -40,9 +40,11 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 FP4_PER_BF16 = 4.0                                 # nominal dense ratio 9 / 2.25 PFLOP/s
 WORKLOAD = ("mlp_fwd_bwd: tokens 8192, hidden 5120, ffn 20480, up -> relu^2 -> down; "
             "6 NVFP4 GEMMs + 12 NVFP4 operands (8 single quantisations, 2 dual-orientation ones for the "
-            "weights; RHT+SR on Wgrad operands) + 2 relu^2 kernels")
+            "weights; RHT+SR on Wgrad operands) + 2 relu^2 kernels that also return max|out| for the next "
+            "rowwise quantisation")
 QUANT_BYTES_SINGLE = 4.5625   # bf16, two passes: read 2 + 2, write 0.5 + 1/16 bytes per element
 QUANT_BYTES_DUAL = 5.125      # bf16, two passes, two outputs: read 2 + 2, write 2 x (0.5 + 1/16)
+QUANT_BYTES_AMAX_IN = 2.5625  # bf16, amax supplied by the producer: read 2, write 0.5 + 1/16
 
 
 def peaks():
@@ -129,6 +131,8 @@ class MlpStep:
         self.ws = B.workspace(max(B.nvfp4_linear_workspace_size(M_TOK, FFN, HID),
                                   B.nvfp4_linear_workspace_size(M_TOK, HID, FFN)), device)
         self.qws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), device)
+        self.amax_h = torch.zeros(4, dtype=torch.float32, device=device)    # max|h|, from relu^2
+        self.amax_dy1 = torch.zeros(4, dtype=torch.float32, device=device)  # max|dY1|, from relu^2 bwd
         mk = B.empty_nvfp4
         # NVFP4 operands of the explicit call sequence (same work as linear_fwd/bwd)
         self.q = {
@@ -142,14 +146,15 @@ class MlpStep:
         self.launches = 0
         torch.cuda.synchronize()
 
-    def _quant(self, x, key, colwise=False, sr=False, rht=False, ev=None):
+    def _quant(self, x, key, colwise=False, sr=False, rht=False, amax_in=None, ev=None):
         B = self.B
         B.nvfp4_quantize(x, orientation=B.NVFP4_COLWISE if colwise else B.NVFP4_ROWWISE,
-                         rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, rht=rht, seed=SEED, out=self.q[key],
-                         ws=self.qws)
+                         rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, rht=rht, seed=SEED, amax_in=amax_in,
+                         out=self.q[key], ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
-            ev.append(("quant", x.numel() * QUANT_BYTES_SINGLE, torch.cuda.Event(enable_timing=True)))
+            per_elem = QUANT_BYTES_AMAX_IN if amax_in is not None else QUANT_BYTES_SINGLE
+            ev.append(("quant", x.numel() * per_elem, torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
 
     def _dual(self, x, key_r, key_c, sr=False, rht=False, ev=None):
@@ -183,12 +188,13 @@ class MlpStep:
         self._quant(d["X"], "X_r", ev=ev)
         self._dual(d["W1"], "W1_r", "W1_c", ev=ev)
         self._gemm("X_r", "W1_r", self.Y1, ev)
-        B.nvfp4_relu2_fwd(self.Y1, out=self.h)
+        # relu^2 also returns max|h|, so h's rowwise quantisation skips its amax pass
+        B.nvfp4_relu2_fwd_amax(self.Y1, out=self.h, amax_out=self.amax_h, ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
             ev.append(("relu2", self.Y1.numel(), torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
-        self._quant(self.h, "h_r", ev=ev)
+        self._quant(self.h, "h_r", amax_in=self.amax_h, ev=ev)
         self._dual(d["W2"], "W2_r", "W2_c", ev=ev)
         self._gemm("h_r", "W2_r", self.Y2, ev)
         # down-projection backward: dh = dY2 . W2, dW2 = dY2^T h
@@ -197,13 +203,13 @@ class MlpStep:
         self._quant(d["dY2"], "dY2_c", colwise=True, sr=True, rht=True, ev=ev)
         self._quant(self.h, "h_c", colwise=True, rht=True, ev=ev)
         self._gemm("dY2_c", "h_c", self.dW2, ev)
-        B.nvfp4_relu2_bwd(self.dh, self.Y1, out=self.dY1)
+        B.nvfp4_relu2_bwd_amax(self.dh, self.Y1, out=self.dY1, amax_out=self.amax_dy1, ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
             ev.append(("relu2", self.Y1.numel(), torch.cuda.Event(enable_timing=True)))
             ev[-1][2].record()
         # up-projection backward: dX = dY1 . W1, dW1 = dY1^T X
-        self._quant(self.dY1, "dY1_r", ev=ev)
+        self._quant(self.dY1, "dY1_r", amax_in=self.amax_dy1, ev=ev)
         self._gemm("dY1_r", "W1_c", self.dX, ev)
         self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, ev=ev)
         self._quant(d["X"], "X_c", colwise=True, rht=True, ev=ev)
@@ -421,7 +427,8 @@ def run_ours(args):
             "roofline_quantize": {"bound": "hbm", "kernels": "amax*, quantize_rowwise, quantize_colwise (+dual)",
                                   "achieved": q_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                   "frac": q_gbs / pk["hbm_gbs"],
-                                  "bytes_per_elem": {"single": QUANT_BYTES_SINGLE, "dual": QUANT_BYTES_DUAL},
+                                  "bytes_per_elem": {"single": QUANT_BYTES_SINGLE, "dual": QUANT_BYTES_DUAL,
+                                                     "amax_supplied": QUANT_BYTES_AMAX_IN},
                                   "calls_per_step": q[2] // args.steps, "peak_source": src + " hbm_gbs",
                                   "call_ms": q[0] / q[2]},
             "breakdown_ms_per_step": {k: v[0] / args.steps for k, v in stats.items()},

@@ -218,6 +218,19 @@ NVFP4_API nvfp4_status nvfp4_linear_fwd_noalloc(const void *X, const void *W, vo
 NVFP4_API nvfp4_status nvfp4_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t stream);
 NVFP4_API nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t stream);
 
+/* The same two kernels, also writing max |output| over the n stored bf16
+ * values to *amax_out (device float, 16-byte aligned) -- the amax a
+ * following nvfp4_quantize of the output would compute in its first pass, so
+ * it can be passed there as amax_in and that pass skipped (the pages'
+ * per-tensor FP32 scale, aisight.pl, section "Architektura NVFP4 kontra
+ * ograniczenia mikroskalowania", is then derived from it unchanged).
+ * workspace: >= nvfp4_quantize_workspace_size() bytes, 16-byte aligned,
+ * device memory (per-CTA partials).  Two launches.  n = 0 writes 0. */
+NVFP4_API nvfp4_status nvfp4_relu2_fwd_amax(const void *y, void *h, int64_t n, float *amax_out, void *workspace,
+                                            size_t ws_bytes, cudaStream_t stream);
+NVFP4_API nvfp4_status nvfp4_relu2_bwd_amax(const void *dh, const void *y, void *dy, int64_t n, float *amax_out,
+                                            void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronise `stream`, then read and clear the workspace's device status
  * word: NVFP4_OK, NVFP4_ERR_DEVICE_TIMEOUT, or NVFP4_ERR_CUDA if the stream
  * reports an error. */

@@ -34,7 +34,8 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_gemm", "nvfp4_linear_workspace_size", "nvfp4_linear_fwd", "nvfp4_linear_bwd",
            "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
            "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
-           "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual")
+           "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
+           "nvfp4_relu2_bwd_amax")
 
 
 class CTensor(C.Structure):
@@ -79,6 +80,8 @@ def load():
         "nvfp4_selftest_wait_timeout": (i32, [vp, sz, u64, vp]),
         "nvfp4_quantize_dual_workspace_size": (sz, []),
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
+        "nvfp4_relu2_fwd_amax": (i32, [vp, vp, i64, vp, vp, sz, vp]),
+        "nvfp4_relu2_bwd_amax": (i32, [vp, vp, vp, i64, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -250,6 +253,26 @@ def nvfp4_relu2_bwd(dh, y, out=None, stream=None):
     out = out if out is not None else torch.empty_like(y)
     _ok(load().nvfp4_relu2_bwd(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _stream(stream)), "nvfp4_relu2_bwd")
     return out
+
+
+def nvfp4_relu2_fwd_amax(y, out=None, amax_out=None, ws=None, stream=None):
+    """relu(y)^2 and max |output| (a 1-element float32 CUDA tensor); returns (out, amax_out)."""
+    out = out if out is not None else torch.empty_like(y)
+    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), y.device)
+    _ok(load().nvfp4_relu2_fwd_amax(_ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "nvfp4_relu2_fwd_amax")
+    return out, amax_out
+
+
+def nvfp4_relu2_bwd_amax(dh, y, out=None, amax_out=None, ws=None, stream=None):
+    """dh * 2 relu(y) and max |output|; returns (out, amax_out)."""
+    out = out if out is not None else torch.empty_like(y)
+    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), y.device)
+    _ok(load().nvfp4_relu2_bwd_amax(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "nvfp4_relu2_bwd_amax")
+    return out, amax_out
 
 
 def nvfp4_check(ws, stream=None):

@@ -362,7 +362,7 @@ nvfp4_status nvfp4_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t str
     if (!aligned16(y) || !aligned16(h)) return NVFP4_ERR_ALIGNMENT;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-    return call.done(from_cuda(launch_relu2_fwd(y, h, n, stream, &call.launches)));
+    return call.done(from_cuda(launch_relu2_fwd(y, h, n, nullptr, nullptr, stream, &call.launches)));
 }
 
 nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t stream) {
@@ -373,7 +373,36 @@ nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n,
     if (!aligned16(dh) || !aligned16(y) || !aligned16(dy)) return NVFP4_ERR_ALIGNMENT;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-    return call.done(from_cuda(launch_relu2_bwd(dh, y, dy, n, stream, &call.launches)));
+    return call.done(from_cuda(launch_relu2_bwd(dh, y, dy, n, nullptr, nullptr, stream, &call.launches)));
+}
+
+nvfp4_status nvfp4_relu2_fwd_amax(const void *y, void *h, int64_t n, float *amax_out, void *workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    Call call;
+    if (n < 0) return NVFP4_ERR_SHAPE;
+    if (!amax_out || (n > 0 && (!y || !h))) return NVFP4_ERR_INVALID_ARG;
+    if ((n > 0 && (!aligned16(y) || !aligned16(h))) || !aligned16(amax_out)) return NVFP4_ERR_ALIGNMENT;
+    if (!workspace || ws_bytes < kQuantizeWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    return call.done(from_cuda(launch_relu2_fwd(y, h, n, amax_out, partials, stream, &call.launches)));
+}
+
+nvfp4_status nvfp4_relu2_bwd_amax(const void *dh, const void *y, void *dy, int64_t n, float *amax_out,
+                                  void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    Call call;
+    if (n < 0) return NVFP4_ERR_SHAPE;
+    if (!amax_out || (n > 0 && (!dh || !y || !dy))) return NVFP4_ERR_INVALID_ARG;
+    if ((n > 0 && (!aligned16(dh) || !aligned16(y) || !aligned16(dy))) || !aligned16(amax_out))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!workspace || ws_bytes < kQuantizeWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    return call.done(from_cuda(launch_relu2_bwd(dh, y, dy, n, amax_out, partials, stream, &call.launches)));
 }
 
 nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream) {

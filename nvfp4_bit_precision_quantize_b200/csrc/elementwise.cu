@@ -1,7 +1,10 @@
 // elementwise.cu -- squared-ReLU activation of the MLP block and its derivative.
 //   h  = relu(y) * relu(y)       dy = dh * (2 * relu(y))
 // one binary32 operation each, then bf16 round-to-nearest-even; relu(y) is +0
-// for y <= 0.  16-byte vectors (8 bf16) per thread, grid-stride.
+// for y <= 0.  16-byte vectors (8 bf16) per thread, grid-stride.  The AMAX
+// variants also return max |output| (of the stored bf16 values), one partial
+// per CTA reduced by a second one-CTA kernel, so that the NVFP4 quantisation
+// that follows can skip its own amax pass (tensor scale from a supplied amax).
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,54 +30,111 @@ __device__ __forceinline__ uint32_t drelu2_pair(uint32_t dh, uint32_t y) {
     return pack_bf16x2(__fmul_rn(bf16lo(dh), ga), __fmul_rn(bf16hi(dh), gb));
 }
 
+__device__ __forceinline__ float absmax_pair(float m, uint32_t w) {
+    return fmaxf(m, fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w))));
+}
+// Block-wide max written as this CTA's partial.
+__device__ __forceinline__ void write_partial(float m, float *partials) {
+    __shared__ float s_red[kThreads / 32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = 0.0f;
+        for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
+        partials[blockIdx.x] = b;
+    }
+}
+
+template <bool AMAX>
 __global__ void __launch_bounds__(kThreads) relu2_fwd_kernel(const uint16_t *__restrict__ y, uint16_t *__restrict__ h,
-                                                             int64_t n) {
+                                                             int64_t n, float *__restrict__ partials) {
     const int64_t nv = n / 8, stride = (int64_t)gridDim.x * kThreads;
+    float m = 0.0f;
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nv; i += stride) {
         const uint4 v = ldg_stream(y + 8 * i);
-        reinterpret_cast<uint4 *>(h)[i] = make_uint4(relu2_pair(v.x), relu2_pair(v.y), relu2_pair(v.z), relu2_pair(v.w));
+        const uint4 o = make_uint4(relu2_pair(v.x), relu2_pair(v.y), relu2_pair(v.z), relu2_pair(v.w));
+        reinterpret_cast<uint4 *>(h)[i] = o;
+        if (AMAX) m = absmax_pair(absmax_pair(absmax_pair(absmax_pair(m, o.x), o.y), o.z), o.w);
     }
     for (int64_t i = 8 * nv + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
         const float a = relu(__uint_as_float((uint32_t)y[i] << 16));
-        h[i] = bf16_of(__fmul_rn(a, a));
+        const uint16_t o = bf16_of(__fmul_rn(a, a));
+        h[i] = o;
+        if (AMAX) m = fmaxf(m, fabsf(__uint_as_float((uint32_t)o << 16)));
     }
+    if (AMAX) write_partial(m, partials);
 }
 
+template <bool AMAX>
 __global__ void __launch_bounds__(kThreads) relu2_bwd_kernel(const uint16_t *__restrict__ dh,
                                                              const uint16_t *__restrict__ y, uint16_t *__restrict__ dy,
-                                                             int64_t n) {
+                                                             int64_t n, float *__restrict__ partials) {
     const int64_t nv = n / 8, stride = (int64_t)gridDim.x * kThreads;
+    float m = 0.0f;
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nv; i += stride) {
         const uint4 g = ldg_stream(dh + 8 * i), v = ldg_stream(y + 8 * i);
-        reinterpret_cast<uint4 *>(dy)[i] =
+        const uint4 o =
             make_uint4(drelu2_pair(g.x, v.x), drelu2_pair(g.y, v.y), drelu2_pair(g.z, v.z), drelu2_pair(g.w, v.w));
+        reinterpret_cast<uint4 *>(dy)[i] = o;
+        if (AMAX) m = absmax_pair(absmax_pair(absmax_pair(absmax_pair(m, o.x), o.y), o.z), o.w);
     }
     for (int64_t i = 8 * nv + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
         const float g = __fmul_rn(2.0f, relu(__uint_as_float((uint32_t)y[i] << 16)));
-        dy[i] = bf16_of(__fmul_rn(__uint_as_float((uint32_t)dh[i] << 16), g));
+        const uint16_t o = bf16_of(__fmul_rn(__uint_as_float((uint32_t)dh[i] << 16), g));
+        dy[i] = o;
+        if (AMAX) m = fmaxf(m, fabsf(__uint_as_float((uint32_t)o << 16)));
     }
+    if (AMAX) write_partial(m, partials);
 }
 
-unsigned grid_for(int64_t n) {
+// max over the partials -> *out (one CTA)
+__global__ void __launch_bounds__(kThreads) amax_reduce_kernel(const float *__restrict__ partials, int count,
+                                                               float *__restrict__ out) {
+    __shared__ float s_red[kThreads / 32];
+    const float m = reduce_partials_max(partials, count, s_red);
+    if (threadIdx.x == 0) *out = m;
+}
+
+unsigned grid_for(int64_t n, int64_t cap_ctas) {
     const int64_t want = (n / 8 + kThreads - 1) / kThreads;
-    const int64_t cap = 8LL * num_sms();
-    return (unsigned)std::max<int64_t>(1, std::min(want, cap));
+    return (unsigned)std::max<int64_t>(1, std::min(want, cap_ctas));
 }
 
 }  // namespace
 
-cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t s, int *launches) {
-    if (n == 0) return cudaSuccess;
-    relu2_fwd_kernel<<<grid_for(n), kThreads, 0, s>>>(static_cast<const uint16_t *>(y), static_cast<uint16_t *>(h), n);
-    ++*launches;
+cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, float *amax_out, float *partials, cudaStream_t s,
+                             int *launches) {
+    const uint16_t *yy = static_cast<const uint16_t *>(y);
+    uint16_t *hh = static_cast<uint16_t *>(h);
+    if (!amax_out) {
+        if (n == 0) return cudaSuccess;
+        relu2_fwd_kernel<false><<<grid_for(n, 8LL * num_sms()), kThreads, 0, s>>>(yy, hh, n, nullptr);
+        ++*launches;
+        return cudaGetLastError();
+    }
+    const unsigned grid = grid_for(n, std::min<int64_t>(4LL * num_sms(), kMaxPartials));
+    relu2_fwd_kernel<true><<<grid, kThreads, 0, s>>>(yy, hh, n, partials);
+    amax_reduce_kernel<<<1, kThreads, 0, s>>>(partials, (int)grid, amax_out);
+    *launches += 2;
     return cudaGetLastError();
 }
 
-cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t s, int *launches) {
-    if (n == 0) return cudaSuccess;
-    relu2_bwd_kernel<<<grid_for(n), kThreads, 0, s>>>(static_cast<const uint16_t *>(dh),
-                                                       static_cast<const uint16_t *>(y), static_cast<uint16_t *>(dy), n);
-    ++*launches;
+cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, float *amax_out, float *partials,
+                             cudaStream_t s, int *launches) {
+    const uint16_t *gg = static_cast<const uint16_t *>(dh), *yy = static_cast<const uint16_t *>(y);
+    uint16_t *dd = static_cast<uint16_t *>(dy);
+    if (!amax_out) {
+        if (n == 0) return cudaSuccess;
+        relu2_bwd_kernel<false><<<grid_for(n, 8LL * num_sms()), kThreads, 0, s>>>(gg, yy, dd, n, nullptr);
+        ++*launches;
+        return cudaGetLastError();
+    }
+    const unsigned grid = grid_for(n, std::min<int64_t>(4LL * num_sms(), kMaxPartials));
+    relu2_bwd_kernel<true><<<grid, kThreads, 0, s>>>(gg, yy, dd, n, partials);
+    amax_reduce_kernel<<<1, kThreads, 0, s>>>(partials, (int)grid, amax_out);
+    *launches += 2;
     return cudaGetLastError();
 }
 

@@ -55,9 +55,11 @@ struct GemmArgs {
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches);
-cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t s, int *launches);
-cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t s,
+// amax_out (optional): max |output| written there; partials: kMaxPartials floats when amax_out is set.
+cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, float *amax_out, float *partials, cudaStream_t s,
                              int *launches);
+cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, float *amax_out, float *partials,
+                             cudaStream_t s, int *launches);
 
 // One bounded wait on an mbarrier nothing arrives on; records the timeout status.
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);

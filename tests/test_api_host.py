@@ -142,3 +142,14 @@ def test_quantize_dual_rejections(lib):
     assert dual(wsb=4352) == binding.NVFP4_ERR_WORKSPACE              # single-orientation size is not enough
     assert dual(w=None) == binding.NVFP4_ERR_WORKSPACE
     assert dual(x=0x10008) == binding.NVFP4_ERR_ALIGNMENT
+
+
+def test_relu2_amax_rejections(lib):
+    ws, a = C.c_void_p(0x20000), C.c_void_p(0x30000)
+    y, h = C.c_void_p(0x10000), C.c_void_p(0x40000)
+    assert lib.nvfp4_relu2_fwd_amax(y, h, -1, a, ws, 1 << 20, None) == binding.NVFP4_ERR_SHAPE
+    assert lib.nvfp4_relu2_fwd_amax(y, h, 64, None, ws, 1 << 20, None) == binding.NVFP4_ERR_INVALID_ARG
+    assert lib.nvfp4_relu2_fwd_amax(y, h, 64, C.c_void_p(0x30004), ws, 1 << 20, None) == binding.NVFP4_ERR_ALIGNMENT
+    assert lib.nvfp4_relu2_fwd_amax(y, h, 64, a, ws, 100, None) == binding.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_relu2_bwd_amax(y, y, h, 64, a, None, 1 << 20, None) == binding.NVFP4_ERR_WORKSPACE
+    assert lib.nvfp4_relu2_bwd_amax(None, y, h, 64, a, ws, 1 << 20, None) == binding.NVFP4_ERR_INVALID_ARG

@@ -8,7 +8,7 @@ import oracle
 from nvfp4_bit_precision_quantize_b200 import binding as B
 from nvfp4_bit_precision_quantize_b200 import workloads as W
 
-from gpu_helpers import assert_gemm_close, to_dev
+from gpu_helpers import assert_gemm_close, check_quantize, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -99,3 +99,27 @@ def test_mlp_block_reduced(cuda_lib):
     for got, ref_t in ((Y2, Y2f), (dW2, dY2f.T @ hf), (dX, dY1f @ W1f), (dW1, dY1f.T @ Xf)):
         rel = (torch.linalg.norm(got.float() - ref_t) / torch.linalg.norm(ref_t)).item()
         assert np.isfinite(rel) and rel < 0.35, rel
+
+
+@pytest.mark.parametrize("n", [0, 8, 1000, 4096 + 3, 1 << 20])
+def test_relu2_amax_variants(n, cuda_lib):
+    """The amax variants store the same bf16 outputs as the plain kernels and return
+    max |output| exactly; a quantisation given that amax equals one that computes it."""
+    rng = np.random.default_rng(n + 3)
+    y = W.bf16_bits(rng.standard_normal(n).astype(np.float32) * np.float32(3.0))
+    dh = W.bf16_bits(rng.standard_normal(n).astype(np.float32))
+    yd, dhd = to_dev(y), to_dev(dh)
+    h, ah = B.nvfp4_relu2_fwd_amax(yd)
+    g, ag = B.nvfp4_relu2_bwd_amax(dhd, yd)
+    torch.cuda.synchronize()
+    hb = h.view(torch.int16).cpu().numpy().view(np.uint16)
+    gb = g.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(hb, oracle.relu2_fwd(y))
+    assert np.array_equal(gb, oracle.relu2_bwd(dh, y))
+    f = lambda b: np.abs((b.astype(np.uint32) << 16).view(np.float32))  # noqa: E731
+    assert ah[0].item() == (float(f(hb).max()) if n else 0.0)
+    assert ag[0].item() == (float(f(gb).max()) if n else 0.0)
+    if n and n % 64 == 0 and n >= 4096:
+        x = hb.reshape(-1, 64)
+        check_quantize(x, amax_in=ah[0].item())
+        check_quantize(gb.reshape(-1, 64), amax_in=ag[0].item())
