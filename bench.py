@@ -45,6 +45,7 @@ WORKLOAD = ("mlp_fwd_bwd: tokens 8192, hidden 5120, ffn 20480, up -> relu^2 -> d
 QUANT_BYTES_SINGLE = 4.5625   # bf16, two passes: read 2 + 2, write 0.5 + 1/16 bytes per element
 QUANT_BYTES_DUAL = 5.125      # bf16, two passes, two outputs: read 2 + 2, write 2 x (0.5 + 1/16)
 QUANT_BYTES_AMAX_IN = 2.5625  # bf16, amax supplied by the producer: read 2, write 0.5 + 1/16
+MX_BYTES = 2.53125            # bf16 MXFP4: read 2, write 0.5 + 1/32
 
 
 def peaks():
@@ -397,6 +398,20 @@ def run_ours(args):
     e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
     B.nvfp4_check(step.ws)
 
+    # MXFP4 (the pages' comparison format) rowwise quantisation of the step's h, timed apart
+    # from the step: one pass, 2 B read + 0.5 + 1/32 B written per element
+    mx_out = B.nvfp4_quantize_mx(step.h)
+    for _ in range(3):
+        B.nvfp4_quantize_mx(step.h, out=mx_out)
+    torch.cuda.synchronize()
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    m0.record()
+    for _ in range(20):
+        B.nvfp4_quantize_mx(step.h, out=mx_out)
+    m1.record()
+    torch.cuda.synchronize()
+    mx_us = m0.elapsed_time(m1) / 20 * 1e3
+
     pk, src = peaks()
     if rank == 0:
         g = stats["gemm"]
@@ -431,6 +446,11 @@ def run_ours(args):
                                                      "amax_supplied": QUANT_BYTES_AMAX_IN},
                                   "calls_per_step": q[2] // args.steps, "peak_source": src + " hbm_gbs",
                                   "call_ms": q[0] / q[2]},
+            "mxfp4_quantize": {"tensor": "h %dx%d bf16, rowwise" % tuple(step.h.shape), "us_per_call": mx_us,
+                               "achieved": step.h.numel() * MX_BYTES / (mx_us * 1e-6) / 1e9, "unit": "GB/s",
+                               "peak": pk["hbm_gbs"],
+                               "frac": step.h.numel() * MX_BYTES / (mx_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                               "bytes_per_elem": MX_BYTES},
             "breakdown_ms_per_step": {k: v[0] / args.steps for k, v in stats.items()},
             "e2e": {"value": nproc * GEMM_FLOPS / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -35,7 +35,7 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
            "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
-           "nvfp4_relu2_bwd_amax")
+           "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx")
 
 
 class CTensor(C.Structure):
@@ -82,6 +82,8 @@ def load():
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
         "nvfp4_relu2_fwd_amax": (i32, [vp, vp, i64, vp, vp, sz, vp]),
         "nvfp4_relu2_bwd_amax": (i32, [vp, vp, vp, i64, vp, vp, sz, vp]),
+        "nvfp4_mx_scales_bytes": (sz, [i64, i64]),
+        "nvfp4_quantize_mx": (i32, [vp, i32, i64, i64, i64, tp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -128,8 +130,8 @@ class NVFP4Tensor:
     k: int
 
     def c(self):
-        return CTensor(self.codes.data_ptr(), self.scales.data_ptr(), self.tensor_scale.data_ptr(),
-                       self.rows, self.k)
+        ts = self.tensor_scale.data_ptr() if self.tensor_scale is not None else None  # MXFP4 has none
+        return CTensor(self.codes.data_ptr(), self.scales.data_ptr(), ts, self.rows, self.k)
 
 
 def nvfp4_codes_bytes(rows, k):
@@ -173,6 +175,23 @@ def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, 
                                int(bool(rht)), seed, _ptr(amax_in), C.byref(ct), _ptr(ws), ws.numel(),
                                _stream(stream))
     _ok(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_mx_scales_bytes(rows, k):
+    return load().nvfp4_mx_scales_bytes(rows, k)
+
+
+def nvfp4_quantize_mx(x, out=None, stream=None):
+    """MXFP4 rowwise quantisation of a 2-D float32/bfloat16 CUDA tensor (C % 32 == 0)."""
+    R, Cc = x.shape
+    out = out or NVFP4Tensor(codes=torch.empty((R, Cc // 2), dtype=torch.uint8, device=x.device),
+                             scales=torch.empty(max(nvfp4_mx_scales_bytes(R, Cc), 16), dtype=torch.uint8,
+                                                device=x.device),
+                             tensor_scale=None, rows=R, k=Cc)
+    ct = out.c()
+    _ok(load().nvfp4_quantize_mx(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), C.byref(ct), _stream(stream)),
+        "nvfp4_quantize_mx")
     return out
 
 

@@ -492,6 +492,108 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4, rowwise, one pass (no tensor scale): blocks of 32 along the columns,
+// E8M0 scale 2^X with X = floor(log2 amax_b) - 2 clamped to [-127, 127], each
+// element E2M1(v * 2^-X) by round-to-nearest-even.  Same persistent walk and
+// 64-row tiles as the NVFP4 rowwise pass; a block spans 32/N lanes of a row.
+// Scales use the 128x4 atom order with four 32-blocks per atom word.
+// ---------------------------------------------------------------------------
+struct MxParams {
+    const void *x;
+    int64_t R, C, ld;
+    uint8_t *codes;
+    uint8_t *scales;
+};
+
+// E8M0 code of a block amax (finite, >= 0): the biased exponent field minus 2
+// is floor(log2 amax) - 2 + 127; fields 0..2 (zero, subnormal, tiny) clamp to 0.
+__device__ __forceinline__ uint32_t mx_code(float amax) {
+    const uint32_t ef = __float_as_uint(amax) >> 23;
+    return ef >= 2u ? ef - 2u : 0u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const MxParams p) {
+    constexpr int N = Vec<T>::N;
+    constexpr int LPB = 32 / N;          // lanes per 32-block
+    constexpr int TILE_C = 32 * N;
+    constexpr int TILE_R = 64;
+    constexpr int RPW = TILE_R / (kThreads / 32);
+    constexpr int ATOMS = TILE_C / 128;  // scale atoms per tile row band
+    __shared__ __align__(16) uint8_t s_sc[ATOMS * 512];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *x = static_cast<const T *>(p.x);
+    const int64_t K = p.C;
+    const int64_t KB4 = (K + 127) / 128;
+    const int64_t tiles_c = (p.C + TILE_C - 1) / TILE_C;
+    const int64_t tiles_r = 2 * ((p.R + 127) / 128);
+    const int64_t ntiles = tiles_c * tiles_r;
+
+    auto load = [&](int64_t t, uint4(&buf)[RPW]) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t c = tc * TILE_C + lane * N;
+        const int64_t r0 = tr * TILE_R + warp * RPW;
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
+            const int64_t r = r0 + i;
+            buf[i] = (c < p.C && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+
+    int64_t t = ntiles - 1 - (int64_t)blockIdx.x;
+    uint4 cur[RPW], nxt[RPW];
+    if (t >= 0) load(t, cur);
+    for (; t >= 0; t -= gridDim.x) {
+        const int64_t tn = t - gridDim.x;
+        if (tn >= 0) load(tn, nxt);
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t c = tc * TILE_C + lane * N;
+        const bool col_ok = c < p.C;
+        const int half = (int)(tr & 1);
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) {
+            const int rl = warp * RPW + i;
+            const int64_t r = tr * TILE_R + rl;
+            float v[N];
+            Vec<T>::unpack(cur[i], v);
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+#pragma unroll
+            for (int o = 1; o < LPB; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            const uint32_t code = mx_code(m);
+            const float inv = __uint_as_float((254u - code) << 23);  // 2^-X
+            float q[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) q[j] = __fmul_rn(v[j], inv);
+            if (col_ok && r < p.R) {
+                uint8_t *dst = p.codes + r * (K / 2) + c / 2;
+                if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
+                else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+            }
+            if ((lane % LPB) == 0) {
+                const int ra = half * TILE_R + rl, bl = lane / LPB;  // 32-block within the tile
+                s_sc[(bl >> 2) * 512 + (ra & 31) * 16 + ((ra >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)code;
+            }
+        }
+        __syncthreads();
+        const int64_t atom0 = tc * ATOMS;
+        for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
+            const int atom = i >> 5;
+            if (atom0 + atom < KB4) {
+                const int off = atom * 512 + (i & 31) * 16 + 8 * half;
+                uint8_t *dst = p.scales + ((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half;
+                *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(s_sc + off);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < RPW; ++i) cur[i] = nxt[i];
+    }
+}
+
 // Empty tensor: only the tensor scale is defined.
 __global__ void tensor_scale_only_kernel(const float *amax_in, float *tensor_scale) {
     *tensor_scale = tensor_scale_from_amax(amax_in ? *amax_in : 0.0f);
@@ -582,6 +684,19 @@ cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int 
         return cudaGetLastError();
     }
     return a.bf16 ? run_dual<uint16_t>(a, s, launches) : run_dual<float>(a, s, launches);
+}
+
+cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, uint8_t *codes,
+                               uint8_t *scales, cudaStream_t s, int *launches) {
+    if (R == 0 || C == 0) return cudaSuccess;
+    const MxParams p{x, R, C, ld, codes, scales};
+    const int N = bf16 ? Vec<uint16_t>::N : Vec<float>::N;
+    const int64_t tiles = ((C + 32 * N - 1) / (32 * N)) * 2 * ((R + 127) / 128);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
+    if (bf16) quantize_rowwise_mx_kernel<uint16_t><<<grid, kThreads, 0, s>>>(p);
+    else quantize_rowwise_mx_kernel<float><<<grid, kThreads, 0, s>>>(p);
+    ++*launches;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches) {

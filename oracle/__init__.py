@@ -58,6 +58,12 @@ def lib():
         L.oracle_amax.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_int,
                                   C.c_int, C.c_uint64]
         L.oracle_amax.restype = C.c_float
+        L.oracle_e8m0_value.argtypes = [C.c_uint]
+        L.oracle_e8m0_value.restype = C.c_double
+        L.oracle_mx_scale.argtypes = [C.c_float]
+        L.oracle_mx_scale.restype = C.c_uint
+        L.oracle_quantize_mx.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, u8p, u8p]
+        L.oracle_quantize_mx.restype = C.c_int
         L.oracle_quantize_rows.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64,
                                            C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_float,
                                            i64p, C.c_int64, u8p, u8p]
@@ -276,3 +282,42 @@ def relu2_bwd(dh_bits, y_bits):
     out = np.zeros_like(y)
     lib().oracle_relu2_bwd(_p(dh, C.c_uint16), _p(y, C.c_uint16), y.size, _p(out, C.c_uint16))
     return out
+
+
+def e8m0_value(code):
+    return lib().oracle_e8m0_value(int(code))
+
+
+def mx_scale(amax_b):
+    return lib().oracle_mx_scale(float(amax_b))
+
+
+def quantize_mx(x):
+    """MXFP4 rowwise quantisation of a 2-D array (float32, or uint16 bf16 bits), C % 32 == 0.
+
+    Returns (codes [R x C/2] uint8, scales [R x C/32] uint8 E8M0 codes, plain row-major)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        bf16 = 1
+    elif x.dtype == np.float32:
+        bf16 = 0
+    else:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    R, Cc = x.shape
+    codes = np.zeros((R, Cc // 2), np.uint8)
+    scales = np.zeros((R, Cc // 32), np.uint8)
+    if lib().oracle_quantize_mx(x.ctypes.data_as(C.c_void_p), bf16, R, Cc, Cc, _p(codes, C.c_uint8),
+                                _p(scales, C.c_uint8)) != 0:
+        raise ValueError("oracle_quantize_mx rejected the arguments")
+    return codes, scales
+
+
+def dequantize_mx(codes, scales):
+    """Binary64 values of an MXFP4 tensor (plain scales)."""
+    R = codes.shape[0]
+    vals = np.array([lib().oracle_e2m1_value(c) for c in range(16)])
+    lo, hi = codes & 0xF, codes >> 4
+    q = np.empty((R, codes.shape[1] * 2))
+    q[:, 0::2], q[:, 1::2] = vals[lo], vals[hi]
+    sc = np.array([lib().oracle_e8m0_value(int(c)) for c in range(256)])[scales]
+    return q * np.repeat(sc, 32, axis=1)

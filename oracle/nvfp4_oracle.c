@@ -44,6 +44,9 @@
  *                     storage ratio, tensor-scale bounds, SR unbiasedness
  *   gemm / dot        pinned: exact small-integer case vs numpy, brute force
  *   relu2             pinned: torch CPU float32 ops and bf16 cast
+ *   mx (MXFP4)        pinned: E8M0 values, shared exponent on binade
+ *                     boundaries, exact round trip of every E2M1 code at many
+ *                     exponents, saturation, the RTN error bound
  *   Readings (tensor-scale constant 2688, the R8 counter mapping, the sign
  *   word of the Hadamard diagonal, multiply-by-reciprocal) are fixed by this
  *   file, not by the pages: "parity unpinned" for those choices themselves.
@@ -392,6 +395,61 @@ int oracle_quantize_rows(const void *x, int dtype_bf16, int64_t R, int64_t C, in
     for (int64_t i = 0; i < n; ++i)
         quantize_row(x, dtype_bf16, ld, colwise, sr, rht, d, seed, s_t, out_rows[i], K,
                      codes + i * (K / 2), scales + i * (K / 16));
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4, the comparison format of [AIS "Architektura NVFP4 kontra           */
+/* ograniczenia mikroskalowania"]: blocks of 32 elements, one power-of-two   */
+/* scale per block, no per-tensor scale.                                      */
+/* ------------------------------------------------------------------------ */
+
+/* E8M0: an unsigned biased exponent, value 2^(code - 127); 0xFF is NaN. */
+double oracle_e8m0_value(unsigned code)
+{
+    return code == 0xFFu ? NAN : ldexp(1.0, (int)code - 127);
+}
+
+/* Reading of the MX block scale (the pages name the format, not the rule; this
+ * is the OCP Microscaling conversion): shared exponent X = floor(log2 amax_b)
+ * - 2, where 2 is the exponent of E2M1's top binade (6 = 1.5 * 2^2), clamped
+ * to [-127, 127]; amax_b = 0 gives X = -127.  Returns the E8M0 code X + 127. */
+unsigned oracle_mx_scale(float amax_b)
+{
+    if (amax_b == 0.0f) return 0u;
+    int e;
+    frexpf(amax_b, &e);          /* amax_b = f * 2^e, f in [0.5, 1): floor(log2) = e - 1 */
+    int x = (e - 1) - 2;
+    if (x < -127) x = -127;
+    if (x > 127) x = 127;
+    return (unsigned)(x + 127);
+}
+
+/* MXFP4 rowwise quantisation of an [R x C] tensor (C % 32 == 0): codes packed
+ * as for NVFP4 (element 2i in the low nibble), scales plain [R x C/32] E8M0
+ * codes.  Each element is E2M1(v * 2^-X) with round-to-nearest-even,
+ * saturating at 6; the power-of-two product is exact (it can only lose bits
+ * below 2^-126, where every value rounds to zero anyway).  Returns 0, or -1
+ * on bad arguments. */
+int oracle_quantize_mx(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t ld,
+                       uint8_t *codes, uint8_t *scales)
+{
+    if (C % 32 != 0 || R < 0 || C < 0) return -1;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t b = 0; b < C / 32; ++b) {
+            float v[32], amax = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                v[j] = load_in(x, dtype_bf16, ld, r, b * 32 + j);
+                if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
+            }
+            unsigned code = oracle_mx_scale(amax);
+            float inv = ldexpf(1.0f, 127 - (int)code);   /* 2^-X */
+            scales[r * (C / 32) + b] = (uint8_t)code;
+            for (int j = 0; j < 32; j += 2) {
+                unsigned lo = oracle_e2m1_rtn(v[j] * inv), hi = oracle_e2m1_rtn(v[j + 1] * inv);
+                codes[r * (C / 2) + (b * 32 + j) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
     return 0;
 }
 
