@@ -40,8 +40,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 FP4_PER_BF16 = 4.0                                 # nominal dense ratio 9 / 2.25 PFLOP/s
 WORKLOAD = ("mlp_fwd_bwd: tokens 8192, hidden 5120, ffn 20480, up -> relu^2 -> down; "
             "6 NVFP4 GEMMs + 12 NVFP4 operands (8 single quantisations, 2 dual-orientation ones for the "
-            "weights; RHT+SR on Wgrad operands) + 2 relu^2 kernels that also return max|out| for the next "
-            "rowwise quantisation")
+            "weights; RHT+SR on Wgrad operands) + 2 relu^2 kernels that also return max|out| and max|RHT(out)| "
+            "for the two quantisations of their output")
 QUANT_BYTES_SINGLE = 4.5625   # bf16, two passes: read 2 + 2, write 0.5 + 1/16 bytes per element
 QUANT_BYTES_DUAL = 5.125      # bf16, two passes, two outputs: read 2 + 2, write 2 x (0.5 + 1/16)
 QUANT_BYTES_AMAX_IN = 2.5625  # bf16, amax supplied by the producer: read 2, write 0.5 + 1/16
@@ -134,6 +134,8 @@ class MlpStep:
         self.qws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), device)
         self.amax_h = torch.zeros(4, dtype=torch.float32, device=device)    # max|h|, from relu^2
         self.amax_dy1 = torch.zeros(4, dtype=torch.float32, device=device)  # max|dY1|, from relu^2 bwd
+        self.amax_h_rht = torch.zeros(4, dtype=torch.float32, device=device)     # max|RHT(h)|
+        self.amax_dy1_rht = torch.zeros(4, dtype=torch.float32, device=device)   # max|RHT(dY1)|
         mk = B.empty_nvfp4
         # NVFP4 operands of the explicit call sequence (same work as linear_fwd/bwd)
         self.q = {
@@ -189,8 +191,9 @@ class MlpStep:
         self._quant(d["X"], "X_r", ev=ev)
         self._dual(d["W1"], "W1_r", "W1_c", ev=ev)
         self._gemm("X_r", "W1_r", self.Y1, ev)
-        # relu^2 also returns max|h|, so h's rowwise quantisation skips its amax pass
-        B.nvfp4_relu2_fwd_amax(self.Y1, out=self.h, amax_out=self.amax_h, ws=self.qws)
+        # relu^2 also returns max|h| and max|RHT(h)|, so both quantisations of h skip their amax pass
+        B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=SEED, out=self.h, amax_out=self.amax_h,
+                                   amax_rht_out=self.amax_h_rht, ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
             ev.append(("relu2", self.Y1.numel(), torch.cuda.Event(enable_timing=True)))
@@ -202,9 +205,10 @@ class MlpStep:
         self._quant(d["dY2"], "dY2_r", ev=ev)
         self._gemm("dY2_r", "W2_c", self.dh, ev)
         self._quant(d["dY2"], "dY2_c", colwise=True, sr=True, rht=True, ev=ev)
-        self._quant(self.h, "h_c", colwise=True, rht=True, ev=ev)
+        self._quant(self.h, "h_c", colwise=True, rht=True, amax_in=self.amax_h_rht, ev=ev)
         self._gemm("dY2_c", "h_c", self.dW2, ev)
-        B.nvfp4_relu2_bwd_amax(self.dh, self.Y1, out=self.dY1, amax_out=self.amax_dy1, ws=self.qws)
+        B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=SEED, out=self.dY1, amax_out=self.amax_dy1,
+                                   amax_rht_out=self.amax_dy1_rht, ws=self.qws)
         self.launches += B.nvfp4_last_launch_count()
         if ev is not None:
             ev.append(("relu2", self.Y1.numel(), torch.cuda.Event(enable_timing=True)))
@@ -212,7 +216,7 @@ class MlpStep:
         # up-projection backward: dX = dY1 . W1, dW1 = dY1^T X
         self._quant(self.dY1, "dY1_r", amax_in=self.amax_dy1, ev=ev)
         self._gemm("dY1_r", "W1_c", self.dX, ev)
-        self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, ev=ev)
+        self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, amax_in=self.amax_dy1_rht, ev=ev)
         self._quant(d["X"], "X_c", colwise=True, rht=True, ev=ev)
         self._gemm("dY1_c", "X_c", self.dW1, ev)
         dp.allreduce_grads([self.dW1, self.dW2])

@@ -250,6 +250,22 @@ NVFP4_API nvfp4_status nvfp4_relu2_fwd_amax(const void *y, void *h, int64_t n, f
 NVFP4_API nvfp4_status nvfp4_relu2_bwd_amax(const void *dh, const void *y, void *dy, int64_t n, float *amax_out,
                                             void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* The same outputs over a contiguous [R x C] bf16 tensor (R % 16 == 0,
+ * C % 8 == 0), writing both amax values the two quantisations of the output
+ * need: *amax_out = max |out| (rowwise) and *amax_rht_out = max |RHT(out)|,
+ * the 16-point random Hadamard transform with the signs of `seed` applied down
+ * each column's 16-row groups -- the amax nvfp4_quantize(out, NVFP4_COLWISE,
+ * ..., rht = 1, seed) computes in its first pass (transform on the Wgrad
+ * operands: aisight.pl, section "Technologie stabilizujace proces
+ * treningowy").  workspace: >= nvfp4_quantize_dual_workspace_size() bytes,
+ * 16-byte aligned.  Two launches. */
+NVFP4_API nvfp4_status nvfp4_relu2_fwd_amax_rht(const void *y, void *h, int64_t R, int64_t C, uint64_t seed,
+                                                float *amax_out, float *amax_rht_out, void *workspace,
+                                                size_t ws_bytes, cudaStream_t stream);
+NVFP4_API nvfp4_status nvfp4_relu2_bwd_amax_rht(const void *dh, const void *y, void *dy, int64_t R, int64_t C,
+                                                uint64_t seed, float *amax_out, float *amax_rht_out,
+                                                void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronise `stream`, then read and clear the workspace's device status
  * word: NVFP4_OK, NVFP4_ERR_DEVICE_TIMEOUT, or NVFP4_ERR_CUDA if the stream
  * reports an error. */

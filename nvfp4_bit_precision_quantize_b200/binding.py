@@ -35,7 +35,8 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_relu2_fwd", "nvfp4_relu2_bwd", "nvfp4_check", "nvfp4_last_launch_count",
            "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
-           "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx")
+           "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
+           "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht")
 
 
 class CTensor(C.Structure):
@@ -84,6 +85,8 @@ def load():
         "nvfp4_relu2_bwd_amax": (i32, [vp, vp, vp, i64, vp, vp, sz, vp]),
         "nvfp4_mx_scales_bytes": (sz, [i64, i64]),
         "nvfp4_quantize_mx": (i32, [vp, i32, i64, i64, i64, tp, vp]),
+        "nvfp4_relu2_fwd_amax_rht": (i32, [vp, vp, i64, i64, u64, vp, vp, vp, sz, vp]),
+        "nvfp4_relu2_bwd_amax_rht": (i32, [vp, vp, vp, i64, i64, u64, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -292,6 +295,33 @@ def nvfp4_relu2_bwd_amax(dh, y, out=None, amax_out=None, ws=None, stream=None):
     _ok(load().nvfp4_relu2_bwd_amax(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), ws.numel(),
                                     _stream(stream)), "nvfp4_relu2_bwd_amax")
     return out, amax_out
+
+
+def nvfp4_relu2_fwd_amax_rht(y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
+    """relu(y)^2 of a 2-D bf16 tensor plus max|out| and max|RHT(out)|; returns (out, amax, amax_rht)."""
+    R, Cc = y.shape
+    out = out if out is not None else torch.empty_like(y)
+    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    amax_rht_out = amax_rht_out if amax_rht_out is not None else torch.empty(4, dtype=torch.float32,
+                                                                             device=y.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), y.device)
+    _ok(load().nvfp4_relu2_fwd_amax_rht(_ptr(y), _ptr(out), R, Cc, seed, _ptr(amax_out), _ptr(amax_rht_out),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "nvfp4_relu2_fwd_amax_rht")
+    return out, amax_out, amax_rht_out
+
+
+def nvfp4_relu2_bwd_amax_rht(dh, y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
+    """dh * 2 relu(y) of 2-D bf16 tensors plus max|out| and max|RHT(out)|; returns (out, amax, amax_rht)."""
+    R, Cc = y.shape
+    out = out if out is not None else torch.empty_like(y)
+    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    amax_rht_out = amax_rht_out if amax_rht_out is not None else torch.empty(4, dtype=torch.float32,
+                                                                             device=y.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), y.device)
+    _ok(load().nvfp4_relu2_bwd_amax_rht(_ptr(dh), _ptr(y), _ptr(out), R, Cc, seed, _ptr(amax_out),
+                                        _ptr(amax_rht_out), _ptr(ws), ws.numel(), _stream(stream)),
+        "nvfp4_relu2_bwd_amax_rht")
+    return out, amax_out, amax_rht_out
 
 
 def nvfp4_check(ws, stream=None):

@@ -427,6 +427,38 @@ nvfp4_status nvfp4_relu2_bwd_amax(const void *dh, const void *y, void *dy, int64
     return call.done(from_cuda(launch_relu2_bwd(dh, y, dy, n, amax_out, partials, stream, &call.launches)));
 }
 
+namespace {
+nvfp4_status relu2_amax_rht_impl(const void *dh, const void *y, void *out, int64_t R, int64_t C, uint64_t seed,
+                                 float *amax_out, float *amax_rht_out, void *workspace, size_t ws_bytes,
+                                 cudaStream_t stream) {
+    Call call;
+    if (R < 0 || C < 0 || R % 16 != 0 || C % 8 != 0) return NVFP4_ERR_SHAPE;
+    if (!amax_out || !amax_rht_out || !y || !out) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out) || (dh && !aligned16(dh)) || !aligned16(amax_out) ||
+        !aligned16(amax_rht_out))
+        return NVFP4_ERR_ALIGNMENT;
+    if (!workspace || ws_bytes < kDualWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    return call.done(from_cuda(launch_relu2_amax_rht(dh, y, out, R, C, seed, amax_out, amax_rht_out, partials,
+                                                     stream, &call.launches)));
+}
+}  // namespace
+
+nvfp4_status nvfp4_relu2_fwd_amax_rht(const void *y, void *h, int64_t R, int64_t C, uint64_t seed, float *amax_out,
+                                      float *amax_rht_out, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    return relu2_amax_rht_impl(nullptr, y, h, R, C, seed, amax_out, amax_rht_out, workspace, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_relu2_bwd_amax_rht(const void *dh, const void *y, void *dy, int64_t R, int64_t C, uint64_t seed,
+                                      float *amax_out, float *amax_rht_out, void *workspace, size_t ws_bytes,
+                                      cudaStream_t stream) {
+    if (!dh) return NVFP4_ERR_INVALID_ARG;
+    return relu2_amax_rht_impl(dh, y, dy, R, C, seed, amax_out, amax_rht_out, workspace, ws_bytes, stream);
+}
+
 nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream) {
     if (!workspace) return NVFP4_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return NVFP4_ERR_CUDA;

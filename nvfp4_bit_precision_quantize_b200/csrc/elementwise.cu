@@ -97,6 +97,71 @@ __global__ void __launch_bounds__(kThreads) amax_reduce_kernel(const float *__re
     if (threadIdx.x == 0) *out = m;
 }
 
+// 2-D variant over a contiguous [R x C] tensor (R % 16 == 0, C % 8 == 0): one
+// work unit = a 16-row group x 4 columns (one 8-byte load per row; a warp's
+// loads cover 256 contiguous bytes of a row), so each column's 16 consecutive
+// outputs sit in one thread and both max |out| and max |RHT(out)| (the 16-point
+// transform down the rows, as the colwise quantiser applies it) come from the
+// values just stored.
+template <bool BWD>
+__global__ void __launch_bounds__(kThreads, 2) relu2_amax_rht_kernel(const uint16_t *__restrict__ dh,
+                                                                     const uint16_t *__restrict__ y,
+                                                                     uint16_t *__restrict__ out, int64_t R, int64_t C,
+                                                                     uint64_t seed, float *__restrict__ partials_plain,
+                                                                     float *__restrict__ partials_rht) {
+    const uint32_t signs = rht_sign_bits(seed);
+    const int64_t chunks = C / 4;
+    const int64_t total = (R / 16) * chunks;
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll 1
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total; u += (int64_t)gridDim.x * kThreads) {
+        const int64_t g = u / chunks, cc = u - g * chunks;
+        const int64_t base = g * 16 * C + cc * 4;
+        uint2 o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(y + base + i * C));
+            if (BWD) {
+                const uint2 gr = __ldg(reinterpret_cast<const uint2 *>(dh + base + i * C));
+                o[i] = make_uint2(drelu2_pair(gr.x, v.x), drelu2_pair(gr.y, v.y));
+            } else {
+                o[i] = make_uint2(relu2_pair(v.x), relu2_pair(v.y));
+            }
+            *reinterpret_cast<uint2 *>(out + base + i * C) = o[i];
+            m0 = absmax_pair(absmax_pair(m0, o[i].x), o[i].y);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float t[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t w = (j >> 1) ? o[i].y : o[i].x;
+                t[i] = (j & 1) ? bf16hi(w) : bf16lo(w);
+            }
+            rht16(t, signs);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m1 = fmaxf(m1, fabsf(t[i]));
+        }
+    }
+    write_partial(m0, partials_plain);
+    __syncthreads();
+    write_partial(m1, partials_rht);
+}
+
+// max over both partial sets -> *out_plain, *out_rht (one CTA)
+__global__ void __launch_bounds__(kThreads) amax_reduce2_kernel(const float *__restrict__ partials_plain,
+                                                                const float *__restrict__ partials_rht, int count,
+                                                                float *__restrict__ out_plain,
+                                                                float *__restrict__ out_rht) {
+    __shared__ float s_red[kThreads / 32];
+    const float a = reduce_partials_max(partials_plain, count, s_red);
+    const float b = reduce_partials_max(partials_rht, count, s_red);
+    if (threadIdx.x == 0) {
+        *out_plain = a;
+        *out_rht = b;
+    }
+}
+
 unsigned grid_for(int64_t n, int64_t cap_ctas) {
     const int64_t want = (n / 8 + kThreads - 1) / kThreads;
     return (unsigned)std::max<int64_t>(1, std::min(want, cap_ctas));
@@ -134,6 +199,29 @@ cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n,
     const unsigned grid = grid_for(n, std::min<int64_t>(4LL * num_sms(), kMaxPartials));
     relu2_bwd_kernel<true><<<grid, kThreads, 0, s>>>(gg, yy, dd, n, partials);
     amax_reduce_kernel<<<1, kThreads, 0, s>>>(partials, (int)grid, amax_out);
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+cudaError_t launch_relu2_amax_rht(const void *dh, const void *y, void *out, int64_t R, int64_t C, uint64_t seed,
+                                  float *amax_out, float *amax_rht_out, float *partials, cudaStream_t s,
+                                  int *launches) {
+    const int64_t units = (R / 16) * (C / 4);
+    const unsigned grid = (unsigned)std::max<int64_t>(
+        1, std::min<int64_t>((units + kThreads - 1) / kThreads, std::min<int64_t>(4LL * num_sms(), kMaxPartials)));
+    const uint16_t *yy = static_cast<const uint16_t *>(y);
+    uint16_t *oo = static_cast<uint16_t *>(out);
+    if (dh)
+        relu2_amax_rht_kernel<true><<<grid, kThreads, 0, s>>>(static_cast<const uint16_t *>(dh), yy, oo, R, C, seed,
+                                                              partials, partials + kMaxPartials);
+    else
+        relu2_amax_rht_kernel<false><<<grid, kThreads, 0, s>>>(nullptr, yy, oo, R, C, seed, partials,
+                                                               partials + kMaxPartials);
+    amax_reduce2_kernel<<<1, kThreads, 0, s>>>(partials, partials + kMaxPartials, (int)grid, amax_out, amax_rht_out);
     *launches += 2;
     return cudaGetLastError();
 }

@@ -66,6 +66,13 @@ cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n,
 // One bounded wait on an mbarrier nothing arrives on; records the timeout status.
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);
 
+// relu^2 (dh == nullptr) or its derivative over a contiguous [R x C] bf16 tensor (R % 16 == 0,
+// C % 8 == 0), also writing max |out| and max |RHT(out)| (transform down 16-row groups);
+// partials: 2 * kMaxPartials floats.
+cudaError_t launch_relu2_amax_rht(const void *dh, const void *y, void *out, int64_t R, int64_t C, uint64_t seed,
+                                  float *amax_out, float *amax_rht_out, float *partials, cudaStream_t s,
+                                  int *launches);
+
 int num_sms();  // SM count of the current device (cached)
 
 }  // namespace nvfp4

@@ -167,3 +167,15 @@ def test_quantize_mx_rejections(lib):
     assert q(ld=60) == binding.NVFP4_ERR_SHAPE
     assert q(x=0x10008) == binding.NVFP4_ERR_ALIGNMENT
     assert lib.nvfp4_quantize_mx(C.c_void_p(0x10000), 1, 64, 64, 64, None, None) == binding.NVFP4_ERR_INVALID_ARG
+
+
+def test_relu2_amax_rht_rejections(lib):
+    ws, a, b = C.c_void_p(0x20000), C.c_void_p(0x30000), C.c_void_p(0x30010)
+    y, h = C.c_void_p(0x10000), C.c_void_p(0x40000)
+    f = lib.nvfp4_relu2_fwd_amax_rht
+    assert f(y, h, 24, 64, 1, a, b, ws, 1 << 20, None) == binding.NVFP4_ERR_SHAPE       # R % 16
+    assert f(y, h, 32, 60, 1, a, b, ws, 1 << 20, None) == binding.NVFP4_ERR_SHAPE       # C % 8
+    assert f(y, h, 32, 64, 1, a, None, ws, 1 << 20, None) == binding.NVFP4_ERR_INVALID_ARG
+    assert f(y, h, 32, 64, 1, a, b, ws, 4352, None) == binding.NVFP4_ERR_WORKSPACE       # needs two partial sets
+    assert lib.nvfp4_relu2_bwd_amax_rht(None, y, h, 32, 64, 1, a, b, ws, 1 << 20, None) == \
+        binding.NVFP4_ERR_INVALID_ARG

@@ -123,3 +123,28 @@ def test_relu2_amax_variants(n, cuda_lib):
         x = hb.reshape(-1, 64)
         check_quantize(x, amax_in=ah[0].item())
         check_quantize(gb.reshape(-1, 64), amax_in=ag[0].item())
+
+
+@pytest.mark.parametrize("shape", [(16, 8), (48, 200), (512, 392), (8192, 2048)])
+def test_relu2_amax_rht_variants(shape, cuda_lib):
+    """The 2-D variants store the oracle's relu^2 outputs and return max|out| and the
+    colwise Hadamard amax exactly; colwise RHT quantisation given that amax equals the
+    one that computes it."""
+    rng = np.random.default_rng(shape[0] + shape[1])
+    y = W.bf16_bits(rng.standard_normal(shape).astype(np.float32) * np.float32(3.0))
+    dh = W.bf16_bits(rng.standard_normal(shape).astype(np.float32) * np.float32(0.01))
+    yd, dhd = to_dev(y), to_dev(dh)
+    h, ah, ahr = B.nvfp4_relu2_fwd_amax_rht(yd, seed=77)
+    g, ag, agr = B.nvfp4_relu2_bwd_amax_rht(dhd, yd, seed=77)
+    torch.cuda.synchronize()
+    hb = h.view(torch.int16).cpu().numpy().view(np.uint16)
+    gb = g.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(hb, oracle.relu2_fwd(y.ravel()).reshape(shape))
+    assert np.array_equal(gb, oracle.relu2_bwd(dh.ravel(), y.ravel()).reshape(shape))
+    f = lambda b: np.abs((b.astype(np.uint32) << 16).view(np.float32))  # noqa: E731
+    assert ah[0].item() == float(f(hb).max()) and ag[0].item() == float(f(gb).max())
+    assert ahr[0].item() == float(oracle.amax(hb, colwise=True, rht=True, seed=77))
+    assert agr[0].item() == float(oracle.amax(gb, colwise=True, rht=True, seed=77))
+    if shape[0] <= 512:
+        check_quantize(hb, colwise=True, rht=True, seed=77, amax_in=ahr[0].item())
+        check_quantize(gb, colwise=True, sr=True, rht=True, seed=77, amax_in=agr[0].item())
