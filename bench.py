@@ -503,6 +503,11 @@ def run_profile_case(case):
         q = None
         for _ in range(3):
             q = B.nvfp4_quantize(x, out=q, ws=ws, seed=SEED, **kw)
+    elif case == "quant_mx":  # MXFP4 rowwise of an h-shaped tensor
+        x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, FFN)))).to(dev)
+        q = None
+        for _ in range(3):
+            q = B.nvfp4_quantize_mx(x, out=q)
     elif case == "quant_dual":  # the step's dY1: rowwise RTN + colwise RHT + SR from one read
         x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, FFN), 1e-3))).to(dev)
         ws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), dev)
@@ -523,7 +528,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy", "quant_dual"],
+    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy", "quant_dual", "quant_mx"],
                     help="run one kernel a few times for an ncu capture instead of the benchmark")
     args = ap.parse_args()
     if args.profile_case:
