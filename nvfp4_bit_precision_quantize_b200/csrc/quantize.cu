@@ -322,9 +322,11 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
 // owns rows 32w..32w+31 (two 16-row groups) and each lane N adjacent columns,
 // so every block (one column x 16 rows) sits in one thread's registers: the
 // transform, block amax and encoding need no shuffles.  A lane's 16 code bytes
-// per column (two groups) form one 16-byte unit, staged in shared memory with
-// an xor swizzle so both the scatter and the row-contiguous read-out are free
-// of bank conflicts beyond the 4-wavefront minimum.
+// per column (two groups) form one 16-byte unit in shared memory (each group
+// writes its 8-byte half as soon as it is encoded), placed with an xor swizzle
+// so both the scatter and the row-contiguous read-out are free of bank
+// conflicts beyond the 4-wavefront minimum.  The DUAL variant also encodes the
+// rowwise (RTN) blocks of the same rows from the same registers.
 // ---------------------------------------------------------------------------
 template <typename T, bool SR, bool RHT, bool DUAL>
 __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QParams p) {
