@@ -10,7 +10,8 @@ gradients are summed over NCCL (weak scaling).
 
 Prints one JSON line.  `value` = GEMM FLOPs of all ranks / device step time
 (max over ranks).  `e2e` = the same through the public calls with pinned host
-inputs copied in and the block output copied back every step.  `--impl
+inputs copied in and the block output copied back every step (on copy streams,
+double-buffered, overlapping the neighbouring steps' compute).  `--impl
 reference` times the CPU oracle on a bounded sample of the same step instead.
 """
 import argparse
@@ -221,22 +222,72 @@ class MlpStep:
         self._gemm("dY1_c", "X_c", self.dW1, ev)
         dp.allreduce_grads([self.dW1, self.dW2])
 
-    def public_step(self):
+    def public_step(self, X=None, dY2=None, Y2=None):
         """The same step through the composite public calls (linear_fwd/bwd, relu2)."""
         B, d = self.B, self.d
-        B.nvfp4_linear_fwd(d["X"], d["W1"], out=self.Y1, ws=self.ws)
+        X = d["X"] if X is None else X
+        dY2 = d["dY2"] if dY2 is None else dY2
+        Y2 = self.Y2 if Y2 is None else Y2
+        B.nvfp4_linear_fwd(X, d["W1"], out=self.Y1, ws=self.ws)
         self.launches += B.nvfp4_last_launch_count()
         B.nvfp4_relu2_fwd(self.Y1, out=self.h)
         self.launches += B.nvfp4_last_launch_count()
-        B.nvfp4_linear_fwd(self.h, d["W2"], out=self.Y2, ws=self.ws)
+        B.nvfp4_linear_fwd(self.h, d["W2"], out=Y2, ws=self.ws)
         self.launches += B.nvfp4_last_launch_count()
-        B.nvfp4_linear_bwd(d["dY2"], self.h, d["W2"], seed=SEED, dX=self.dh, dW=self.dW2, ws=self.ws)
+        B.nvfp4_linear_bwd(dY2, self.h, d["W2"], seed=SEED, dX=self.dh, dW=self.dW2, ws=self.ws)
         self.launches += B.nvfp4_last_launch_count()
         B.nvfp4_relu2_bwd(self.dh, self.Y1, out=self.dY1)
         self.launches += B.nvfp4_last_launch_count()
-        B.nvfp4_linear_bwd(self.dY1, d["X"], d["W1"], seed=SEED, dX=self.dX, dW=self.dW1, ws=self.ws)
+        B.nvfp4_linear_bwd(self.dY1, X, d["W1"], seed=SEED, dX=self.dX, dW=self.dW1, ws=self.ws)
         self.launches += B.nvfp4_last_launch_count()
         dp.allreduce_grads([self.dW1, self.dW2])
+
+
+class E2EPipeline:
+    """Steps through the public calls with every step's host->device input copy and
+    device->host output copy on their own streams, double-buffered, so that step i+1's
+    inputs arrive and step i-1's output leaves while step i computes (a training loop's
+    prefetch).  Every step still moves its own bytes inside the timed region."""
+
+    def __init__(self, step):
+        self.step = step
+        self.xs = [step.d["X"], torch.empty_like(step.d["X"])]
+        self.dys = [step.d["dY2"], torch.empty_like(step.d["dY2"])]
+        self.y2s = [step.Y2, torch.empty_like(step.Y2)]
+        self.y2_host = [torch.empty(step.Y2.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(self, n):
+        st, comp = self.step, torch.cuda.current_stream()
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_ready, done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+        def load(b):
+            with torch.cuda.stream(self.s_in):
+                self.xs[b].copy_(st.host["X"], non_blocking=True)
+                self.dys[b].copy_(st.host["dY2"], non_blocking=True)
+                in_ready[b].record(self.s_in)
+
+        self.s_in.wait_stream(comp)
+        self.s_out.wait_stream(comp)
+        load(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                if i >= 1:
+                    self.s_in.wait_event(done[1 - b])  # step i-1 no longer reads buffer 1-b
+                load(1 - b)
+            comp.wait_event(in_ready[b])
+            if i >= 2:
+                comp.wait_event(out_done[b])           # step i-2's output has left buffer b
+            st.public_step(self.xs[b], self.dys[b], self.y2s[b])
+            done[b].record(comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(done[b])
+                self.y2_host[b].copy_(self.y2s[b], non_blocking=True)
+                out_done[b].record(self.s_out)
+        comp.wait_stream(self.s_out)
+        comp.wait_stream(self.s_in)
 
 
 def kernel_stats(events_per_step):
@@ -380,22 +431,17 @@ def run_ours(args):
     B.nvfp4_check(step.ws)
     stats = kernel_stats(events)
 
-    # end to end through the public calls: pinned host inputs in, block output out
+    # end to end through the public calls: pinned host inputs in, block output out, every step
     h2d = step.host["X"].numel() * 2 + step.host["dY2"].numel() * 2
-    y2_host = torch.empty(step.Y2.shape, dtype=torch.bfloat16).pin_memory()
-    d2h = y2_host.numel() * 2
-    for _ in range(2):
-        step.public_step()
+    d2h = step.Y2.numel() * 2
+    pipe = E2EPipeline(step)
+    pipe.run(3)
     dp.barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
-        step.d["X"].copy_(step.host["X"], non_blocking=True)
-        step.d["dY2"].copy_(step.host["dY2"], non_blocking=True)
-        step.public_step()
-        y2_host.copy_(step.Y2, non_blocking=True)
+    pipe.run(args.steps)
     e1.record()
     torch.cuda.synchronize()
     dp.barrier()
