@@ -119,21 +119,25 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t 
 /* MXFP4, the comparison format of aisight.pl, section "Architektura NVFP4
  * kontra ograniczenia mikroskalowania": blocks of 32 elements along the
  * contiguous dim (rowwise), one E8M0 (power-of-two) scale per block, no
- * per-tensor scale.  Scale 2^X with X = floor(log2 amax_b) - 2 (2 is the
+ * per-tensor scale, in either orientation (as for nvfp4_quantize: colwise
+ * blocks run down the rows and the output is the transpose).  Scale 2^X with
+ * X = floor(log2 amax_b) - 2 (2 is the
  * exponent of E2M1's top binade), clamped to [-127, 127], X = -127 for an
  * all-zero block; each element is E2M1(v * 2^-X), round to nearest even,
  * saturating at +-6 (the OCP Microscaling conversion; the pages name the
  * format only).  One pass over x, no workspace.
- * x: [R x C] dtype, row stride ld elements, 16-byte aligned, C % 32 == 0.
- * out: rows = R, k = C; codes R*C/2 bytes as for NVFP4 (element 2i in the
- * low nibble); scales nvfp4_mx_scales_bytes(R, C) bytes of E8M0 codes in the
+ * x: [R x C] dtype, row stride ld elements, 16-byte aligned; rowwise needs
+ * C % 32 == 0, colwise R % 32 == 0 and C * element size % 16 == 0.
+ * out: [rows' x k] = [R x C] (rowwise) or [C x R] (colwise); codes rows'*k/2
+ * bytes as for NVFP4 (element 2i in the low nibble); scales
+ * nvfp4_mx_scales_bytes(rows', k) bytes of E8M0 codes in the
  * 128x4 atom order of the NVFP4 scales with four 32-blocks per atom word
  * (rows padded to 128, blocks to 4, padding 0); out->tensor_scale unused.
  * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_SHAPE, NVFP4_ERR_ALIGNMENT,
  * NVFP4_ERR_UNSUPPORTED_DEVICE, NVFP4_ERR_CUDA. */
 NVFP4_API size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k);
 NVFP4_API nvfp4_status nvfp4_quantize_mx(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
-                                         const nvfp4_tensor *out, cudaStream_t stream);
+                                         int orientation, const nvfp4_tensor *out, cudaStream_t stream);
 
 /* Both NVFP4 operands of one tensor from one read of it (the layer's
  * backward pass needs dY rowwise for Dgrad and colwise with the Hadamard

@@ -84,7 +84,7 @@ def load():
         "nvfp4_relu2_fwd_amax": (i32, [vp, vp, i64, vp, vp, sz, vp]),
         "nvfp4_relu2_bwd_amax": (i32, [vp, vp, vp, i64, vp, vp, sz, vp]),
         "nvfp4_mx_scales_bytes": (sz, [i64, i64]),
-        "nvfp4_quantize_mx": (i32, [vp, i32, i64, i64, i64, tp, vp]),
+        "nvfp4_quantize_mx": (i32, [vp, i32, i64, i64, i64, i32, tp, vp]),
         "nvfp4_relu2_fwd_amax_rht": (i32, [vp, vp, i64, i64, u64, vp, vp, vp, sz, vp]),
         "nvfp4_relu2_bwd_amax_rht": (i32, [vp, vp, vp, i64, i64, u64, vp, vp, vp, sz, vp]),
     }
@@ -185,16 +185,18 @@ def nvfp4_mx_scales_bytes(rows, k):
     return load().nvfp4_mx_scales_bytes(rows, k)
 
 
-def nvfp4_quantize_mx(x, out=None, stream=None):
-    """MXFP4 rowwise quantisation of a 2-D float32/bfloat16 CUDA tensor (C % 32 == 0)."""
+def nvfp4_quantize_mx(x, orientation=NVFP4_ROWWISE, out=None, stream=None):
+    """MXFP4 quantisation of a 2-D float32/bfloat16 CUDA tensor (rowwise: C % 32 == 0;
+    colwise, transposed output: R % 32 == 0)."""
     R, Cc = x.shape
-    out = out or NVFP4Tensor(codes=torch.empty((R, Cc // 2), dtype=torch.uint8, device=x.device),
-                             scales=torch.empty(max(nvfp4_mx_scales_bytes(R, Cc), 16), dtype=torch.uint8,
+    rows, k = (Cc, R) if orientation == NVFP4_COLWISE else (R, Cc)
+    out = out or NVFP4Tensor(codes=torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device),
+                             scales=torch.empty(max(nvfp4_mx_scales_bytes(rows, k), 16), dtype=torch.uint8,
                                                 device=x.device),
-                             tensor_scale=None, rows=R, k=Cc)
+                             tensor_scale=None, rows=rows, k=k)
     ct = out.c()
-    _ok(load().nvfp4_quantize_mx(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), C.byref(ct), _stream(stream)),
-        "nvfp4_quantize_mx")
+    _ok(load().nvfp4_quantize_mx(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), orientation, C.byref(ct),
+                                 _stream(stream)), "nvfp4_quantize_mx")
     return out
 
 

@@ -255,21 +255,25 @@ size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k) {
     return (size_t)((rows + 127) / 128) * 128 * (size_t)((k + 127) / 128) * 4;
 }
 
-nvfp4_status nvfp4_quantize_mx(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
+nvfp4_status nvfp4_quantize_mx(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int orientation,
                                const nvfp4_tensor *out, cudaStream_t stream) {
     Call call;
-    if (!out || !valid_dtype(dtype)) return NVFP4_ERR_INVALID_ARG;
-    if (R < 0 || C < 0 || out->rows != R || out->k != C) return NVFP4_ERR_SHAPE;
+    if (!out || !valid_dtype(dtype) || (orientation != NVFP4_ROWWISE && orientation != NVFP4_COLWISE))
+        return NVFP4_ERR_INVALID_ARG;
+    const bool colwise = orientation == NVFP4_COLWISE;
+    if (R < 0 || C < 0 || out->rows != (colwise ? C : R) || out->k != (colwise ? R : C)) return NVFP4_ERR_SHAPE;
     if (R == 0 || C == 0) return call.done(NVFP4_OK);
     if (!x || !out->codes || !out->scales) return NVFP4_ERR_INVALID_ARG;
-    if (ld < C || C % 32 != 0 || R > (1LL << 31) || C > (1LL << 31)) return NVFP4_ERR_SHAPE;
     const size_t es = esize(dtype);
+    if (ld < C || R > (1LL << 31) || C > (1LL << 31)) return NVFP4_ERR_SHAPE;
+    if (!colwise && C % 32 != 0) return NVFP4_ERR_SHAPE;
+    if (colwise && (R % 32 != 0 || (C * (int64_t)es) % 16 != 0)) return NVFP4_ERR_SHAPE;
     if (!aligned16(x) || (ld * (int64_t)es) % 16 != 0 || !aligned16(out->codes) || !aligned16(out->scales))
         return NVFP4_ERR_ALIGNMENT;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-    return call.done(from_cuda(launch_quantize_mx(x, dtype == NVFP4_DTYPE_BF16, R, C, ld, out->codes, out->scales,
-                                                  stream, &call.launches)));
+    return call.done(from_cuda(launch_quantize_mx(x, dtype == NVFP4_DTYPE_BF16, R, C, ld, colwise, out->codes,
+                                                  out->scales, stream, &call.launches)));
 }
 
 size_t nvfp4_quantize_dual_workspace_size(void) { return kDualWorkspace; }

@@ -54,8 +54,8 @@ struct GemmArgs {
 // Each launcher adds the number of kernels it launched to *launches.
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches);
-cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, uint8_t *codes,
-                               uint8_t *scales, cudaStream_t s, int *launches);
+cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool colwise,
+                               uint8_t *codes, uint8_t *scales, cudaStream_t s, int *launches);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches);
 // amax_out (optional): max |output| written there; partials: kMaxPartials floats when amax_out is set.
 cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, float *amax_out, float *partials, cudaStream_t s,

@@ -596,6 +596,61 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const 
     }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4, colwise (blocks of 32 down the rows; output transposed, [C x R]):
+// each thread holds one 32-row block of 8 / sizeof(T) adjacent columns (one
+// 8-byte load per row), so a column's block is in one thread: amax, E8M0 code
+// and the 32 codes (16 bytes, one store into the output row of that column)
+// need no shuffles.  The grid spans the scale atoms' padded extent (columns to
+// a multiple of 128, rows to a multiple of 128), and threads outside the
+// tensor write the zero padding scales.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) quantize_colwise_mx_kernel(const MxParams p) {
+    constexpr int CPT = 8 / (int)sizeof(T);  // columns per thread
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t c0 = ((int64_t)blockIdx.x * 32 + lane) * CPT;
+    const int64_t r0 = ((int64_t)blockIdx.y * (kThreads / 32) + warp) * 32;
+    const int64_t K = p.R;                     // output k (contiguous) = input rows
+    const int64_t KB4 = (K + 127) / 128;       // scale atoms per 128-row tile of the output
+    const int64_t out_rows_pad = ((p.C + 127) / 128) * 128;
+    if (r0 >= KB4 * 128 || c0 >= out_rows_pad) return;
+    const bool rows_ok = r0 < p.R;             // R % 32 == 0: a block is all in or all out
+    const T *x = static_cast<const T *>(p.x);
+    uint2 raw[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        raw[i] = (rows_ok && c0 < p.C) ? __ldg(reinterpret_cast<const uint2 *>(x + (r0 + i) * p.ld + c0))
+                                       : make_uint2(0u, 0u);
+    const int64_t b = r0 / 32;                 // 32-block index along k
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+        const int64_t c = c0 + j;              // output row
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (sizeof(T) == 2) {
+                const uint32_t w = (j >> 1) ? raw[i].y : raw[i].x;
+                v[i] = (j & 1) ? bf16hi(w) : bf16lo(w);
+            } else {
+                v[i] = __uint_as_float(j ? raw[i].y : raw[i].x);
+            }
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+        const uint32_t code = mx_code(m);      // 0 for padding (all-zero) blocks
+        const float inv = __uint_as_float((254u - code) << 23);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+        if (rows_ok && c < p.C) {
+            const uint4 u = make_uint4(e2m1x8(v), e2m1x8(v + 8), e2m1x8(v + 16), e2m1x8(v + 24));
+            *reinterpret_cast<uint4 *>(p.codes + c * (K / 2) + r0 / 2) = u;
+        }
+        p.scales[((c >> 7) * KB4 + (b >> 2)) * 512 + (c & 31) * 16 + ((c >> 5) & 3) * 4 + (b & 3)] = (uint8_t)code;
+    }
+}
+
 // Empty tensor: only the tensor scale is defined.
 __global__ void tensor_scale_only_kernel(const float *amax_in, float *tensor_scale) {
     *tensor_scale = tensor_scale_from_amax(amax_in ? *amax_in : 0.0f);
@@ -688,10 +743,19 @@ cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int 
     return a.bf16 ? run_dual<uint16_t>(a, s, launches) : run_dual<float>(a, s, launches);
 }
 
-cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, uint8_t *codes,
-                               uint8_t *scales, cudaStream_t s, int *launches) {
+cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool colwise,
+                               uint8_t *codes, uint8_t *scales, cudaStream_t s, int *launches) {
     if (R == 0 || C == 0) return cudaSuccess;
     const MxParams p{x, R, C, ld, codes, scales};
+    if (colwise) {
+        const int cpt = bf16 ? 4 : 2;
+        const int64_t cols_pad = ((C + 127) / 128) * 128, rows_pad = ((R + 127) / 128) * 128;
+        dim3 grid((unsigned)((cols_pad + 32 * cpt - 1) / (32 * cpt)), (unsigned)((rows_pad + 255) / 256));
+        if (bf16) quantize_colwise_mx_kernel<uint16_t><<<grid, kThreads, 0, s>>>(p);
+        else quantize_colwise_mx_kernel<float><<<grid, kThreads, 0, s>>>(p);
+        ++*launches;
+        return cudaGetLastError();
+    }
     const int N = bf16 ? Vec<uint16_t>::N : Vec<float>::N;
     const int64_t tiles = ((C + 32 * N - 1) / (32 * N)) * 2 * ((R + 127) / 128);
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());

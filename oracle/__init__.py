@@ -62,7 +62,7 @@ def lib():
         L.oracle_e8m0_value.restype = C.c_double
         L.oracle_mx_scale.argtypes = [C.c_float]
         L.oracle_mx_scale.restype = C.c_uint
-        L.oracle_quantize_mx.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, u8p, u8p]
+        L.oracle_quantize_mx.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_int, u8p, u8p]
         L.oracle_quantize_mx.restype = C.c_int
         L.oracle_quantize_rows.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64,
                                            C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_float,
@@ -292,10 +292,11 @@ def mx_scale(amax_b):
     return lib().oracle_mx_scale(float(amax_b))
 
 
-def quantize_mx(x):
-    """MXFP4 rowwise quantisation of a 2-D array (float32, or uint16 bf16 bits), C % 32 == 0.
+def quantize_mx(x, colwise=False):
+    """MXFP4 quantisation of a 2-D array (float32, or uint16 bf16 bits); rowwise needs
+    C % 32 == 0, colwise (transposed output) R % 32 == 0.
 
-    Returns (codes [R x C/2] uint8, scales [R x C/32] uint8 E8M0 codes, plain row-major)."""
+    Returns (codes [rows' x K/2] uint8, scales [rows' x K/32] uint8 E8M0 codes, plain row-major)."""
     x = np.ascontiguousarray(x)
     if x.dtype == np.uint16:
         bf16 = 1
@@ -304,9 +305,10 @@ def quantize_mx(x):
     else:
         raise TypeError("x must be float32 or uint16 (bf16 bits)")
     R, Cc = x.shape
-    codes = np.zeros((R, Cc // 2), np.uint8)
-    scales = np.zeros((R, Cc // 32), np.uint8)
-    if lib().oracle_quantize_mx(x.ctypes.data_as(C.c_void_p), bf16, R, Cc, Cc, _p(codes, C.c_uint8),
+    rows, K = (Cc, R) if colwise else (R, Cc)
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, K // 32), np.uint8)
+    if lib().oracle_quantize_mx(x.ctypes.data_as(C.c_void_p), bf16, R, Cc, Cc, int(colwise), _p(codes, C.c_uint8),
                                 _p(scales, C.c_uint8)) != 0:
         raise ValueError("oracle_quantize_mx rejected the arguments")
     return codes, scales

@@ -425,29 +425,32 @@ unsigned oracle_mx_scale(float amax_b)
     return (unsigned)(x + 127);
 }
 
-/* MXFP4 rowwise quantisation of an [R x C] tensor (C % 32 == 0): codes packed
- * as for NVFP4 (element 2i in the low nibble), scales plain [R x C/32] E8M0
- * codes.  Each element is E2M1(v * 2^-X) with round-to-nearest-even,
- * saturating at 6; the power-of-two product is exact (it can only lose bits
- * below 2^-126, where every value rounds to zero anyway).  Returns 0, or -1
- * on bad arguments. */
-int oracle_quantize_mx(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t ld,
+/* MXFP4 quantisation of an [R x C] tensor.  Rowwise (colwise = 0, C % 32 ==
+ * 0): output row o is input row o, blocks run along the columns.  Colwise
+ * (R % 32 == 0): output row o is input column o and blocks run down the rows
+ * (the transposed view, as for NVFP4).  Codes packed as for NVFP4 (element 2i
+ * in the low nibble), scales plain [rows' x K/32] E8M0 codes.  Each element is
+ * E2M1(v * 2^-X) with round-to-nearest-even, saturating at 6; the power-of-two
+ * product is exact (it can only lose bits below 2^-126, where every value
+ * rounds to zero anyway).  Returns 0, or -1 on bad arguments. */
+int oracle_quantize_mx(const void *x, int dtype_bf16, int64_t R, int64_t C, int64_t ld, int colwise,
                        uint8_t *codes, uint8_t *scales)
 {
-    if (C % 32 != 0 || R < 0 || C < 0) return -1;
-    for (int64_t r = 0; r < R; ++r)
-        for (int64_t b = 0; b < C / 32; ++b) {
+    int64_t rows = colwise ? C : R, K = colwise ? R : C;
+    if (K % 32 != 0 || R < 0 || C < 0) return -1;
+    for (int64_t o = 0; o < rows; ++o)
+        for (int64_t b = 0; b < K / 32; ++b) {
             float v[32], amax = 0.0f;
             for (int j = 0; j < 32; ++j) {
-                v[j] = load_in(x, dtype_bf16, ld, r, b * 32 + j);
+                v[j] = colwise ? load_in(x, dtype_bf16, ld, b * 32 + j, o) : load_in(x, dtype_bf16, ld, o, b * 32 + j);
                 if (fabsf(v[j]) > amax) amax = fabsf(v[j]);
             }
             unsigned code = oracle_mx_scale(amax);
             float inv = ldexpf(1.0f, 127 - (int)code);   /* 2^-X */
-            scales[r * (C / 32) + b] = (uint8_t)code;
+            scales[o * (K / 32) + b] = (uint8_t)code;
             for (int j = 0; j < 32; j += 2) {
                 unsigned lo = oracle_e2m1_rtn(v[j] * inv), hi = oracle_e2m1_rtn(v[j + 1] * inv);
-                codes[r * (C / 2) + (b * 32 + j) / 2] = (uint8_t)(lo | (hi << 4));
+                codes[o * (K / 2) + (b * 32 + j) / 2] = (uint8_t)(lo | (hi << 4));
             }
         }
     return 0;

@@ -159,14 +159,18 @@ def test_quantize_mx_rejections(lib):
     assert lib.nvfp4_mx_scales_bytes(1, 32) == 128 * 4
     assert lib.nvfp4_mx_scales_bytes(129, 160) == 256 * 8
     out = _tensor(64, 64)
-    q = lambda x=0x10000, dtype=1, R=64, Cc=64, ld=64, o=out: lib.nvfp4_quantize_mx(  # noqa: E731
-        C.c_void_p(x), dtype, R, Cc, ld, C.byref(o), None)
+    q = lambda x=0x10000, dtype=1, R=64, Cc=64, ld=64, ori=0, o=out: lib.nvfp4_quantize_mx(  # noqa: E731
+        C.c_void_p(x), dtype, R, Cc, ld, ori, C.byref(o), None)
     assert q(dtype=5) == binding.NVFP4_ERR_INVALID_ARG
-    assert q(o=_tensor(64, 48), Cc=48, ld=48) == binding.NVFP4_ERR_SHAPE       # C % 32 != 0
+    assert q(ori=2) == binding.NVFP4_ERR_INVALID_ARG
+    assert q(o=_tensor(64, 48), Cc=48, ld=48) == binding.NVFP4_ERR_SHAPE       # rowwise C % 32 != 0
+    assert q(ori=1, R=48, o=_tensor(64, 48)) == binding.NVFP4_ERR_SHAPE       # colwise R % 32 != 0
+    assert q(ori=1, Cc=68, ld=72, o=_tensor(68, 64)) == binding.NVFP4_ERR_SHAPE  # colwise C * 2 % 16 != 0
     assert q(o=_tensor(32, 64)) == binding.NVFP4_ERR_SHAPE                     # out shape
+    assert q(ori=1, R=96, o=_tensor(96, 64)) == binding.NVFP4_ERR_SHAPE       # colwise out is [C x R]
     assert q(ld=60) == binding.NVFP4_ERR_SHAPE
     assert q(x=0x10008) == binding.NVFP4_ERR_ALIGNMENT
-    assert lib.nvfp4_quantize_mx(C.c_void_p(0x10000), 1, 64, 64, 64, None, None) == binding.NVFP4_ERR_INVALID_ARG
+    assert lib.nvfp4_quantize_mx(C.c_void_p(0x10000), 1, 64, 64, 64, 0, None, None) == binding.NVFP4_ERR_INVALID_ARG
 
 
 def test_relu2_amax_rht_rejections(lib):

@@ -107,3 +107,15 @@ def test_nvfp4_error_below_mxfp4():
         cm, sm = oracle.quantize_mx(x)
         e_mx = np.linalg.norm(oracle.dequantize_mx(cm, sm) - x) / np.linalg.norm(x)
         assert e_nv < e_mx, (name, e_nv, e_mx)
+
+
+def test_colwise_is_rowwise_of_the_transpose():
+    """Colwise MXFP4 of x (blocks down the rows, transposed output) is, by definition of
+    the orientation, the rowwise MXFP4 of x^T."""
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((96, 40)) * np.exp(rng.standard_normal((96, 1)))).astype(np.float32)
+    c1, s1 = oracle.quantize_mx(x, colwise=True)
+    c2, s2 = oracle.quantize_mx(np.ascontiguousarray(x.T))
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    with pytest.raises(ValueError):
+        oracle.quantize_mx(np.zeros((48, 64), np.float32), colwise=True)   # R % 32 != 0
