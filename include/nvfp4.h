@@ -105,7 +105,8 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(void);
  *   [R x C] (out->rows == R, out->k == C).  Requires C % 16 == 0.
  * orientation = NVFP4_COLWISE: blocks run down the R rows and out is the
  *   transpose [C x R] (out->rows == C, out->k == R).  Requires R % 16 == 0
- *   and C a multiple of 8 (bf16) / 4 (f32).
+ *   and C a multiple of 8 (bf16) / 4 (f32), and R <= 65535 * 256.
+ * R and C are at most 2^31.
  * rht != 0 only with NVFP4_COLWISE.  x must be 16-byte aligned and
  * ld * element size a multiple of 16.  workspace: >= nvfp4_quantize_workspace_size()
  * bytes (may be NULL when amax_in is given).  amax_in: optional device float.
@@ -127,7 +128,8 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t 
  * saturating at +-6 (the OCP Microscaling conversion; the pages name the
  * format only).  One pass over x, no workspace.
  * x: [R x C] dtype, row stride ld elements, 16-byte aligned; rowwise needs
- * C % 32 == 0, colwise R % 32 == 0 and C * element size % 16 == 0.
+ * C % 32 == 0, colwise R % 32 == 0, R <= 65535 * 256 and C * element size
+ * % 16 == 0.  R and C are at most 2^31.
  * out: [rows' x k] = [R x C] (rowwise) or [C x R] (colwise); codes rows'*k/2
  * bytes as for NVFP4 (element 2i in the low nibble); scales
  * nvfp4_mx_scales_bytes(rows', k) bytes of E8M0 codes in the
@@ -172,7 +174,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int
  * multiplies by the two tensor scales and writes c_dtype (f32 or bf16,
  * round-to-nearest-even) row-major with leading dimension ldc elements.
  * Requires A->k == B->k, K % 64 == 0, C 16-byte aligned, ldc * element size a
- * multiple of 16.  M or N == 0: nothing is done.  K == 0: C is zero-filled.
+ * multiple of 16, and M, N, K < 2^31.  M or N == 0: nothing is done.
+ * K == 0: C is zero-filled.
  * workspace: >= 256 bytes (status word).
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,

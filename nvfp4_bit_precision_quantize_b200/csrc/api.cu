@@ -73,7 +73,7 @@ nvfp4_status validate_quantize(const void *x, int dtype, int64_t R, int64_t C, i
     if (ld < C) return NVFP4_ERR_SHAPE;
     if (!colwise && C % 16 != 0) return NVFP4_ERR_SHAPE;
     if (colwise && (R % 16 != 0 || (C * (int64_t)es) % 16 != 0)) return NVFP4_ERR_SHAPE;
-    if (R > (1LL << 31) || C > (1LL << 31)) return NVFP4_ERR_SHAPE;
+    if (R > (1LL << 31) || C > (1LL << 31) || (colwise && R > kMaxColwiseRows)) return NVFP4_ERR_SHAPE;
     if (!aligned16(x) || (ld * (int64_t)es) % 16 != 0 || !aligned16(out->codes) || !aligned16(out->scales))
         return NVFP4_ERR_ALIGNMENT;
     if (!amax_in) {
@@ -267,7 +267,7 @@ nvfp4_status nvfp4_quantize_mx(const void *x, nvfp4_dtype dtype, int64_t R, int6
     const size_t es = esize(dtype);
     if (ld < C || R > (1LL << 31) || C > (1LL << 31)) return NVFP4_ERR_SHAPE;
     if (!colwise && C % 32 != 0) return NVFP4_ERR_SHAPE;
-    if (colwise && (R % 32 != 0 || (C * (int64_t)es) % 16 != 0)) return NVFP4_ERR_SHAPE;
+    if (colwise && (R % 32 != 0 || (C * (int64_t)es) % 16 != 0 || R > kMaxColwiseRows)) return NVFP4_ERR_SHAPE;
     if (!aligned16(x) || (ld * (int64_t)es) % 16 != 0 || !aligned16(out->codes) || !aligned16(out->scales))
         return NVFP4_ERR_ALIGNMENT;
     nvfp4_status st = check_device();

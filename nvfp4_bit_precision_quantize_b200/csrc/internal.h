@@ -10,6 +10,9 @@ constexpr int kMaxPartials = 1024;          // per-CTA amax partials in a quanti
 constexpr size_t kStatusBytes = 256;        // status word region at the start of a workspace
 constexpr size_t kQuantizeWorkspace = kStatusBytes + kMaxPartials * sizeof(float);
 constexpr size_t kDualWorkspace = kStatusBytes + 2 * kMaxPartials * sizeof(float);
+// The colwise kernels tile the input rows 256 per grid row, and a grid has at
+// most 65535 rows: the largest R (blocked dim) a colwise quantisation takes.
+constexpr int64_t kMaxColwiseRows = 65535LL * 256;
 
 struct QuantizeArgs {
     const void *x;

@@ -78,6 +78,9 @@ def test_quantize_rejections(lib):
     assert _q(lib, out=_tensor(64, 64, codes=0x1004)) == E.NVFP4_ERR_ALIGNMENT
     assert _q(lib, ws=0) == E.NVFP4_ERR_WORKSPACE
     assert _q(lib, wsb=100) == E.NVFP4_ERR_WORKSPACE
+    big = 65535 * 256 + 16                                            # colwise grid rows run out
+    assert _q(lib, R=big, ld=64, ori=1, out=_tensor(64, big)) == E.NVFP4_ERR_SHAPE
+    assert _q(lib, R=(1 << 31) + 16, Cc=64, out=_tensor((1 << 31) + 16, 64)) == E.NVFP4_ERR_SHAPE
 
 
 def test_gemm_rejections(lib):
@@ -111,6 +114,10 @@ def test_linear_rejections(lib):
         == E.NVFP4_ERR_INVALID_ARG
     assert lib.nvfp4_linear_bwd(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), 100, 128, 128, 1, 1,
                                 1, p(0x6000), ws, None) == E.NVFP4_ERR_SHAPE
+    big = 65535 * 256 + 64                                            # colwise dY / X: R = M too large
+    wsb = lib.nvfp4_linear_workspace_size(big, 128, 128)
+    assert lib.nvfp4_linear_bwd(p(0x1000), p(0x2000), p(0x3000), p(0x4000), p(0x5000), big, 128, 128, 1, 1,
+                                1, p(0x6000), wsb, None) == E.NVFP4_ERR_SHAPE
     assert lib.nvfp4_relu2_fwd(p(0x1001), p(0x2000), 16, None) == E.NVFP4_ERR_ALIGNMENT
     assert lib.nvfp4_relu2_bwd(None, p(0x2000), p(0x3000), 16, None) == E.NVFP4_ERR_INVALID_ARG
 
@@ -170,6 +177,8 @@ def test_quantize_mx_rejections(lib):
     assert q(ori=1, R=96, o=_tensor(96, 64)) == binding.NVFP4_ERR_SHAPE       # colwise out is [C x R]
     assert q(ld=60) == binding.NVFP4_ERR_SHAPE
     assert q(x=0x10008) == binding.NVFP4_ERR_ALIGNMENT
+    big = 65535 * 256 + 32
+    assert q(ori=1, R=big, o=_tensor(64, big)) == binding.NVFP4_ERR_SHAPE      # colwise R limit
     assert lib.nvfp4_quantize_mx(C.c_void_p(0x10000), 1, 64, 64, 64, 0, None, None) == binding.NVFP4_ERR_INVALID_ARG
 
 
