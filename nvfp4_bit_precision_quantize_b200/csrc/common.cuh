@@ -103,18 +103,25 @@ __device__ __forceinline__ uint32_t e2m1x8(const float *v) {
 }
 
 // Stochastic rounding of r onto the E2M1 grid with a 16-bit draw: the
-// magnitude rounds up to the next grid point iff u < frac, u = rnd16 / 2^16.
-// With n = |r| / spacing (exact), ceil(n - u) is exactly that decision.
+// magnitude rounds up to the next grid point iff u < frac, u = rnd16 / 2^16,
+// frac the position of |r| between its two neighbouring grid points.
+// Decided on the binary32 bit pattern.  For |r| >= 1 the grid spacing is the
+// weight of the first mantissa bit, so frac * 2^22 is the low 22 mantissa bits
+// L, and L > rnd16 * 2^6 exactly when L + (2^22 - 1 - rnd16 * 2^6) carries
+// into bit 22; adding that constant and clearing the low 22 bits rounds.
+// For |r| < 1 (spacing 0.5) the same step runs on 1 + |r|, which puts the
+// 0.5-grid on the first mantissa bit; the sum is rounded UP to binary32, which
+// keeps the comparison with the 2^-17-spaced threshold exact (a threshold t on
+// the binary32 grid has x > t iff roundup(x) > t), and 1 is subtracted again
+// (exact).  Values at or above 6 land on 6 or above and are clamped to 6.
 // Returns the exact E2M1 value (sign of r kept), to be encoded by e2m1x*.
 __device__ __forceinline__ float sr_e2m1_value(float r, uint32_t rnd16) {
     const float a = fabsf(r);
-    const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    const float n = __fmul_rn(a, inv_step);
-    const float u = __fsub_rn(__uint_as_float(0x3F800000u | (rnd16 << 7)), 1.0f);
-    const float k = __fadd_rn(ceilf(__fsub_rn(n, u)), 0.0f);
-    float mag = __fmul_rn(k, step);
-    mag = (a >= 6.0f) ? 6.0f : mag;
+    const float base = a < 1.0f ? 1.0f : 0.0f;
+    const float t = __fadd_ru(a, base);
+    const uint32_t carry_in = ((~rnd16 & 0xFFFFu) << 6) | 63u;
+    const float up = __uint_as_float((__float_as_uint(t) + carry_in) & 0xFFC00000u);
+    const float mag = fminf(__fsub_rn(up, base), 6.0f);
     return copysignf(mag, r);
 }
 
