@@ -115,9 +115,9 @@ class ClockSampler:
 class MlpStep:
     """Device buffers and the C-ABI call sequence of one MLP block step."""
 
-    def __init__(self, B, device, seed):
+    def __init__(self, B, device, data_seed=None):
         self.B = B
-        w = W.mlp(seed=seed)
+        w = W.mlp(seed=5, data_seed=data_seed)
         pin = lambda a: W.bits_to_torch_bf16(a).pin_memory()  # noqa: E731
         self.host = {k: pin(v) for k, v in w.items()}
         self.d = {k: v.to(device, non_blocking=True) for k, v in self.host.items()}
@@ -397,7 +397,7 @@ def run_ours(args):
     from nvfp4_bit_precision_quantize_b200 import build as lib_build
     lib_build.build()
     B.load()
-    step = MlpStep(B, device, dp.shard_seed(5, rank))
+    step = MlpStep(B, device, dp.shard_data_seed(5, rank))
 
     # warm-up
     for _ in range(args.warmup):

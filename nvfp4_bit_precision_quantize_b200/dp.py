@@ -29,9 +29,11 @@ def init(backend="nccl", timeout_s=120):
     return ws, rank, local
 
 
-def shard_seed(base_seed, rank):
-    """Data seed of a rank's token shard (distinct shards, same weights)."""
-    return base_seed + 1000 * rank
+def shard_data_seed(base_seed, rank):
+    """Seed of a rank's token shard (its X and dY2; the weights are drawn from
+    base_seed on every rank): None on rank 0, which keeps the single-GPU
+    workload, base_seed + 1000 * rank elsewhere."""
+    return None if rank == 0 else base_seed + 1000 * rank
 
 
 def allreduce_grads(grads):

@@ -83,9 +83,17 @@ def wgrad(seed=4, M=2 * TOKENS, N=FFN, K=HIDDEN):
             "X": bf16_bits(normal(rng, (M, K)))}
 
 
-def mlp(seed=5, M=TOKENS, H=HIDDEN, F=FFN):
+def mlp(seed=5, M=TOKENS, H=HIDDEN, F=FFN, data_seed=None):
+    """The MLP block's inputs.  With data_seed, X and dY2 (a data-parallel
+    rank's token shard) come from their own generator while W1 and W2 stay
+    those of `seed`, so every rank holds the same weights."""
     rng = np.random.default_rng(seed)
-    return {"X": bf16_bits(normal(rng, (M, H))),
-            "W1": bf16_bits(normal(rng, (F, H), 0.02)),
-            "W2": bf16_bits(normal(rng, (H, F), 0.02)),
-            "dY2": bf16_bits(normal(rng, (M, H), 1e-3))}
+    w = {"X": bf16_bits(normal(rng, (M, H))),
+         "W1": bf16_bits(normal(rng, (F, H), 0.02)),
+         "W2": bf16_bits(normal(rng, (H, F), 0.02)),
+         "dY2": bf16_bits(normal(rng, (M, H), 1e-3))}
+    if data_seed is not None:
+        drng = np.random.default_rng(data_seed)
+        w["X"] = bf16_bits(normal(drng, (M, H)))
+        w["dY2"] = bf16_bits(normal(drng, (M, H), 1e-3))
+    return w

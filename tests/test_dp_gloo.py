@@ -1,5 +1,5 @@
 """The data-parallel plumbing (gradient all-reduce, max-over-ranks timing,
-shard seeds) with two gloo ranks on CPU."""
+token shards that share the weights) with two gloo ranks on CPU."""
 import os
 import socket
 
@@ -18,14 +18,15 @@ def _worker(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
                       LOCAL_RANK=str(rank))
     from nvfp4_bit_precision_quantize_b200 import dp
+    from nvfp4_bit_precision_quantize_b200 import workloads as W
     dp.init("gloo", timeout_s=60)
     g1 = torch.full((4, 3), float(rank + 1))
     g2 = torch.arange(6, dtype=torch.float32) * (rank + 1)
     dp.allreduce_grads([g1, g2])
     slowest = dp.max_over_ranks(1.5 + rank)
-    seeds = dp.shard_seed(5, rank)
+    w = W.mlp(seed=5, M=64, H=32, F=48, data_seed=dp.shard_data_seed(5, rank))
     dp.barrier()
-    q.put((rank, g1.tolist(), g2.tolist(), slowest, seeds))
+    q.put((rank, g1.tolist(), g2.tolist(), slowest, {k: v.tolist() for k, v in w.items()}))
     dp.finish()
 
 
@@ -40,8 +41,19 @@ def test_two_rank_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, g1, g2, slowest, seed in res:
+    for rank, g1, g2, slowest, _ in res:
         assert g1 == [[3.0] * 3] * 4
         assert g2 == [float(3 * i) for i in range(6)]
         assert slowest == 2.5
-    assert res[0][4] != res[1][4]
+    w0, w1 = res[0][4], res[1][4]
+    assert w0["W1"] == w1["W1"] and w0["W2"] == w1["W2"]      # one model on every rank
+    assert w0["X"] != w1["X"] and w0["dY2"] != w1["dY2"]      # each rank its own tokens
+
+
+def test_rank0_keeps_the_single_gpu_workload():
+    from nvfp4_bit_precision_quantize_b200 import dp
+    from nvfp4_bit_precision_quantize_b200 import workloads as W
+    a = W.mlp(seed=5, M=64, H=32, F=48)
+    b = W.mlp(seed=5, M=64, H=32, F=48, data_seed=dp.shard_data_seed(5, 0))
+    for k in a:
+        assert (a[k] == b[k]).all(), k
