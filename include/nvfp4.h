@@ -32,6 +32,9 @@
  *     device-side waits record NVFP4_ERR_DEVICE_TIMEOUT there instead of
  *     hanging; nvfp4_check() reads and clears it.
  *   - Non-finite inputs are outside the contract (the result is unspecified).
+ *   - With NVFP4_NVTX=1 in the environment when the process starts, every
+ *     call is wrapped in an NVTX range named after the function, for
+ *     timeline profilers; otherwise no NVTX call is made.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_

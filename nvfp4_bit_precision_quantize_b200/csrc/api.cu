@@ -2,6 +2,9 @@
 // the kernel sequences of the linear layer.  Nothing here allocates memory.
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "internal.h"
 #include "nvfp4.h"
@@ -140,8 +143,28 @@ size_t bwd_bytes(int64_t M, int64_t N, int64_t K) {
     return c.off;
 }
 
-struct Call {  // per-call launch accounting
+// NVTX ranges around the C-ABI calls, for timeline profilers: off unless the
+// process starts with NVFP4_NVTX=1 in its environment (read once).  Without a
+// profiler attached the NVTX calls do nothing.
+bool nvtx_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("NVFP4_NVTX");
+        return e != nullptr && e[0] == '1' && e[1] == '\0';
+    }();
+    return on;
+}
+
+struct Call {  // per-call launch accounting and the optional NVTX range
     int launches = 0;
+    const bool ranged;
+    explicit Call(const char *name) : ranged(nvtx_enabled()) {
+        if (ranged) nvtxRangePushA(name);
+    }
+    ~Call() {
+        if (ranged) nvtxRangePop();
+    }
+    Call(const Call &) = delete;
+    Call &operator=(const Call &) = delete;
     nvfp4_status done(nvfp4_status st) {
         if (st == NVFP4_OK) g_last_launches = launches;
         return st;
@@ -240,7 +263,7 @@ size_t nvfp4_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
 nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int orientation,
                             int rounding, int rht, uint64_t seed, const float *amax_in, const nvfp4_tensor *out,
                             void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     nvfp4_status st =
         validate_quantize(x, dtype, R, C, ld, orientation, rounding, rht, amax_in, out, workspace, ws_bytes);
     if (st != NVFP4_OK) return st;
@@ -257,7 +280,7 @@ size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k) {
 
 nvfp4_status nvfp4_quantize_mx(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int orientation,
                                const nvfp4_tensor *out, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (!out || !valid_dtype(dtype) || (orientation != NVFP4_ROWWISE && orientation != NVFP4_COLWISE))
         return NVFP4_ERR_INVALID_ARG;
     const bool colwise = orientation == NVFP4_COLWISE;
@@ -283,7 +306,7 @@ nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int64_t R, in
                                  const float *amax_col_in, const nvfp4_tensor *out_row,
                                  const nvfp4_tensor *out_col, void *workspace, size_t ws_bytes,
                                  cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     // each orientation's own checks; the dual workspace holds both amax partial sets
     nvfp4_status st = validate_quantize(x, dtype, R, C, ld, NVFP4_ROWWISE, NVFP4_RTN, 0, amax_row_in, out_row,
                                         workspace, ws_bytes);
@@ -300,7 +323,7 @@ nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int64_t R, in
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype, int64_t ldc,
                         void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     nvfp4_status st = validate_gemm(A, B, C, c_dtype, ldc, workspace, ws_bytes);
     if (st != NVFP4_OK) return st;
     if (A->rows == 0 || B->rows == 0) return call.done(NVFP4_OK);  // nothing to launch
@@ -311,7 +334,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, n
 nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
                               nvfp4_dtype dtype, nvfp4_dtype y_dtype, void *workspace, size_t ws_bytes,
                               cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (!valid_dtype(dtype) || !valid_dtype(y_dtype)) return NVFP4_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || K % 64 != 0) return NVFP4_ERR_SHAPE;
     if (M == 0 || N == 0) return call.done(NVFP4_OK);
@@ -340,7 +363,7 @@ nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, 
 nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void *dX, float *dW, int64_t M,
                               int64_t N, int64_t K, nvfp4_dtype dtype, nvfp4_dtype dx_dtype, uint64_t seed,
                               void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (!valid_dtype(dtype) || !valid_dtype(dx_dtype)) return NVFP4_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || M % 64 != 0 || N % 64 != 0 || K % 64 != 0) return NVFP4_ERR_SHAPE;
     if (M == 0 || N == 0 || K == 0) return NVFP4_ERR_SHAPE;
@@ -381,7 +404,7 @@ nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void
 }
 
 nvfp4_status nvfp4_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (n < 0) return NVFP4_ERR_SHAPE;
     if (n == 0) return call.done(NVFP4_OK);
     if (!y || !h) return NVFP4_ERR_INVALID_ARG;
@@ -392,7 +415,7 @@ nvfp4_status nvfp4_relu2_fwd(const void *y, void *h, int64_t n, cudaStream_t str
 }
 
 nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (n < 0) return NVFP4_ERR_SHAPE;
     if (n == 0) return call.done(NVFP4_OK);
     if (!dh || !y || !dy) return NVFP4_ERR_INVALID_ARG;
@@ -404,7 +427,7 @@ nvfp4_status nvfp4_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n,
 
 nvfp4_status nvfp4_relu2_fwd_amax(const void *y, void *h, int64_t n, float *amax_out, void *workspace,
                                   size_t ws_bytes, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (n < 0) return NVFP4_ERR_SHAPE;
     if (!amax_out || (n > 0 && (!y || !h))) return NVFP4_ERR_INVALID_ARG;
     if ((n > 0 && (!aligned16(y) || !aligned16(h))) || !aligned16(amax_out)) return NVFP4_ERR_ALIGNMENT;
@@ -418,7 +441,7 @@ nvfp4_status nvfp4_relu2_fwd_amax(const void *y, void *h, int64_t n, float *amax
 
 nvfp4_status nvfp4_relu2_bwd_amax(const void *dh, const void *y, void *dy, int64_t n, float *amax_out,
                                   void *workspace, size_t ws_bytes, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (n < 0) return NVFP4_ERR_SHAPE;
     if (!amax_out || (n > 0 && (!dh || !y || !dy))) return NVFP4_ERR_INVALID_ARG;
     if ((n > 0 && (!aligned16(dh) || !aligned16(y) || !aligned16(dy))) || !aligned16(amax_out))
@@ -435,7 +458,7 @@ namespace {
 nvfp4_status relu2_amax_rht_impl(const void *dh, const void *y, void *out, int64_t R, int64_t C, uint64_t seed,
                                  float *amax_out, float *amax_rht_out, void *workspace, size_t ws_bytes,
                                  cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (R < 0 || C < 0 || R % 16 != 0 || C % 8 != 0) return NVFP4_ERR_SHAPE;
     if (!amax_out || !amax_rht_out || !y || !out) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(y) || !aligned16(out) || (dh && !aligned16(dh)) || !aligned16(amax_out) ||
@@ -476,7 +499,7 @@ nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream) {
 }
 
 nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_bytes, uint64_t limit_ns, cudaStream_t stream) {
-    Call call;
+    Call call(__func__);
     if (!workspace || ws_bytes < kStatusBytes) return NVFP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
     if (limit_ns == 0 || limit_ns > 2000000000ull) return NVFP4_ERR_INVALID_ARG;

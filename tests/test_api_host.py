@@ -4,6 +4,9 @@ invalid arguments are rejected before anything is launched."""
 import ctypes as C
 import os
 import re
+import subprocess
+import sys
+import textwrap
 
 import pytest
 
@@ -192,3 +195,23 @@ def test_relu2_amax_rht_rejections(lib):
     assert f(y, h, 32, 64, 1, a, b, ws, 4352, None) == binding.NVFP4_ERR_WORKSPACE       # needs two partial sets
     assert lib.nvfp4_relu2_bwd_amax_rht(None, y, h, 32, 64, 1, a, b, ws, 1 << 20, None) == \
         binding.NVFP4_ERR_INVALID_ARG
+
+
+def test_nvtx_ranges_switch_on(lib):
+    """NVFP4_NVTX=1 wraps every call in an NVTX range; with no profiler attached
+    the calls still return their status (here: a rejected flag combination)."""
+    code = textwrap.dedent("""
+        import ctypes as C, sys
+        sys.path.insert(0, %r)
+        from nvfp4_bit_precision_quantize_b200 import binding
+        lib = binding.load()
+        out = binding.CTensor(0x1000, 0x2000, 0x3000, 64, 64)
+        for _ in range(3):
+            st = lib.nvfp4_quantize(C.c_void_p(0x10000), 1, 64, 64, 64, 0, 0, 1, 1, None, C.byref(out),
+                                    C.c_void_p(0x20000), 1 << 20, None)
+        print(st)
+    """ % ROOT)
+    env = dict(os.environ, NVFP4_NVTX="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert int(r.stdout.strip().splitlines()[-1]) == binding.NVFP4_ERR_INVALID_ARG
