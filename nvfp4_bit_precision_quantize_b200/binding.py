@@ -122,6 +122,71 @@ def _ptr(t):
     return C.c_void_p(t.data_ptr()) if t is not None else None
 
 
+# ----------------------------------------------------------------- argument checks
+# The C ABI sees raw pointers and sizes only.  What it cannot check -- that a
+# buffer is device memory of the current device, dense where the call assumes
+# it, of the dtype passed and large enough -- is checked here before the call,
+# so that a wrong tensor raises instead of reaching a kernel.
+
+def _on_device(*tensors):
+    ts = [t for t in tensors if t is not None]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensor on %s: the library takes CUDA tensors" % t.device)
+    if ts:
+        dev = torch.cuda.current_device()
+        for t in ts:
+            if t.device.index != dev:
+                raise ValueError("tensor on %s: the library runs on the current device, cuda:%d" % (t.device, dev))
+
+
+def _dense(name, t, shape=None, dtype=None):
+    """t is contiguous, with the given shape and dtype."""
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s: dtype %s, expected %s" % (name, t.dtype, dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _rows(name, t):
+    """A 2-D tensor whose rows are contiguous (any row stride)."""
+    if t.dim() != 2:
+        raise ValueError("%s must be 2-D, got %d-D" % (name, t.dim()))
+    if t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError("%s: elements of a row must be contiguous (stride(1) == 1)" % name)
+    _dtype_code(t.dtype)
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _scalar_out(name, t):
+    if t is not None and (t.dtype != torch.float32 or t.numel() < 1):
+        raise ValueError("%s must be a float32 tensor with at least one element" % name)
+
+
+def _workspace(ws):
+    if ws is not None and not ws.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    return _nbytes(ws) if ws is not None else 0
+
+
+def _quantised(name, q, scales_bytes):
+    """The buffers of an NVFP4 / MXFP4 tensor are device memory and large enough."""
+    _on_device(q.codes, q.scales, q.tensor_scale)
+    for part, t in (("codes", q.codes), ("scales", q.scales)):
+        if not t.is_contiguous():
+            raise ValueError("%s.%s must be contiguous" % (name, part))
+    if _nbytes(q.codes) < q.rows * (q.k // 2):
+        raise ValueError("%s.codes: %d bytes, need %d" % (name, _nbytes(q.codes), q.rows * (q.k // 2)))
+    if _nbytes(q.scales) < scales_bytes:
+        raise ValueError("%s.scales: %d bytes, need %d" % (name, _nbytes(q.scales), scales_bytes))
+    _scalar_out(name + ".tensor_scale", q.tensor_scale)
+
+
 @dataclass
 class NVFP4Tensor:
     """Device NVFP4 tensor [rows x k]: codes (uint8 [rows, k/2]), scales (uint8,
@@ -169,13 +234,17 @@ def empty_nvfp4(rows, k, device=None):
 def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, seed=1234, amax_in=None,
                    out=None, ws=None, stream=None):
     """Quantise a 2-D float32/bfloat16 CUDA tensor to NVFP4 (see include/nvfp4.h)."""
+    _rows("x", x)
     R, Cc = x.shape
     rows, k = (Cc, R) if orientation == NVFP4_COLWISE else (R, Cc)
     out = out or empty_nvfp4(rows, k, x.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), x.device)
+    _on_device(x, amax_in, ws)
+    _scalar_out("amax_in", amax_in)
+    _quantised("out", out, nvfp4_scales_bytes(out.rows, out.k))
     ct = out.c()
     st = load().nvfp4_quantize(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), orientation, rounding,
-                               int(bool(rht)), seed, _ptr(amax_in), C.byref(ct), _ptr(ws), ws.numel(),
+                               int(bool(rht)), seed, _ptr(amax_in), C.byref(ct), _ptr(ws), _workspace(ws),
                                _stream(stream))
     _ok(st, "nvfp4_quantize")
     return out
@@ -188,12 +257,15 @@ def nvfp4_mx_scales_bytes(rows, k):
 def nvfp4_quantize_mx(x, orientation=NVFP4_ROWWISE, out=None, stream=None):
     """MXFP4 quantisation of a 2-D float32/bfloat16 CUDA tensor (rowwise: C % 32 == 0;
     colwise, transposed output: R % 32 == 0)."""
+    _rows("x", x)
     R, Cc = x.shape
     rows, k = (Cc, R) if orientation == NVFP4_COLWISE else (R, Cc)
     out = out or NVFP4Tensor(codes=torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device),
                              scales=torch.empty(max(nvfp4_mx_scales_bytes(rows, k), 16), dtype=torch.uint8,
                                                 device=x.device),
                              tensor_scale=None, rows=rows, k=k)
+    _on_device(x)
+    _quantised("out", out, nvfp4_mx_scales_bytes(out.rows, out.k))
     ct = out.c()
     _ok(load().nvfp4_quantize_mx(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), orientation, C.byref(ct),
                                  _stream(stream)), "nvfp4_quantize_mx")
@@ -207,14 +279,20 @@ def nvfp4_quantize_dual_workspace_size():
 def nvfp4_quantize_dual(x, col_rounding=NVFP4_RTN, col_rht=False, seed=1234, amax_row_in=None, amax_col_in=None,
                         out_row=None, out_col=None, ws=None, stream=None):
     """Rowwise (RTN) and colwise NVFP4 of one 2-D tensor from one read; returns (row, col)."""
+    _rows("x", x)
     R, Cc = x.shape
     out_row = out_row or empty_nvfp4(R, Cc, x.device)
     out_col = out_col or empty_nvfp4(Cc, R, x.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), x.device)
+    _on_device(x, amax_row_in, amax_col_in, ws)
+    _scalar_out("amax_row_in", amax_row_in)
+    _scalar_out("amax_col_in", amax_col_in)
+    _quantised("out_row", out_row, nvfp4_scales_bytes(out_row.rows, out_row.k))
+    _quantised("out_col", out_col, nvfp4_scales_bytes(out_col.rows, out_col.k))
     cr, cc = out_row.c(), out_col.c()
     st = load().nvfp4_quantize_dual(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), col_rounding,
                                     int(bool(col_rht)), seed, _ptr(amax_row_in), _ptr(amax_col_in), C.byref(cr),
-                                    C.byref(cc), _ptr(ws), ws.numel(), _stream(stream))
+                                    C.byref(cc), _ptr(ws), _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_quantize_dual")
     return out_row, out_col
 
@@ -224,32 +302,53 @@ def nvfp4_gemm(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
     M, N = A.rows, B.rows
     out = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=A.codes.device)
     ws = ws if ws is not None else workspace(256, A.codes.device)
+    _quantised("A", A, nvfp4_scales_bytes(A.rows, A.k))
+    _quantised("B", B, nvfp4_scales_bytes(B.rows, B.k))
+    _rows("out", out)
+    if out.shape[0] < M or out.shape[1] < N:
+        raise ValueError("out: shape %s, need at least (%d, %d)" % (tuple(out.shape), M, N))
+    _on_device(out, ws)
     ca, cb = A.c(), B.c()
     st = load().nvfp4_gemm(C.byref(ca), C.byref(cb), _ptr(out), _dtype_code(out.dtype), out.stride(0), _ptr(ws),
-                           ws.numel(), _stream(stream))
+                           _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_gemm")
     return out
 
 
-def nvfp4_linear_fwd(X, W, y_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+def _linear_operands(X, W):
+    """X [M x K] and W [N x K], contiguous, one dtype; returns (M, N, K)."""
+    _rows("X", X)
+    _rows("W", W)
     M, K = X.shape
     N = W.shape[0]
+    _dense("X", X)
+    _dense("W", W, shape=(N, K), dtype=X.dtype)
+    return M, N, K
+
+
+def nvfp4_linear_fwd(X, W, y_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+    M, N, K = _linear_operands(X, W)
     out = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
     ws = ws if ws is not None else workspace(nvfp4_linear_workspace_size(M, N, K), X.device)
+    _dense("out", out, shape=(M, N))
+    _on_device(X, W, out, ws)
     st = load().nvfp4_linear_fwd(_ptr(X), _ptr(W), _ptr(out), M, N, K, _dtype_code(X.dtype),
-                                 _dtype_code(out.dtype), _ptr(ws), ws.numel(), _stream(stream))
+                                 _dtype_code(out.dtype), _ptr(ws), _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_linear_fwd")
     return out
 
 
 def nvfp4_linear_bwd(dY, X, W, seed=1234, dx_dtype=torch.bfloat16, dX=None, dW=None, ws=None, stream=None):
-    M, N = dY.shape
-    K = X.shape[1]
+    M, N, K = _linear_operands(X, W)
+    _dense("dY", dY, shape=(M, N), dtype=X.dtype)
     dX = dX if dX is not None else torch.empty((M, K), dtype=dx_dtype, device=X.device)
     dW = dW if dW is not None else torch.empty((N, K), dtype=torch.float32, device=X.device)
     ws = ws if ws is not None else workspace(nvfp4_linear_workspace_size(M, N, K), X.device)
+    _dense("dX", dX, shape=(M, K))
+    _dense("dW", dW, shape=(N, K), dtype=torch.float32)
+    _on_device(dY, X, W, dX, dW, ws)
     st = load().nvfp4_linear_bwd(_ptr(dY), _ptr(X), _ptr(W), _ptr(dX), _ptr(dW), M, N, K, _dtype_code(X.dtype),
-                                 _dtype_code(dX.dtype), seed, _ptr(ws), ws.numel(), _stream(stream))
+                                 _dtype_code(dX.dtype), seed, _ptr(ws), _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_linear_bwd")
     return dX, dW
 
@@ -258,82 +357,116 @@ def nvfp4_linear_fwd_noalloc(X, W, y_dtype=torch.bfloat16, out=None, stream=None
     """nvfp4_linear_fwd without a workspace: the library's fixed scratch buffer is
     used instead (see include/nvfp4.h).  Only `out` may be allocated here, and only
     when the caller passes none."""
-    M, K = X.shape
-    N = W.shape[0]
+    M, N, K = _linear_operands(X, W)
     out = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
+    _dense("out", out, shape=(M, N))
+    _on_device(X, W, out)
     st = load().nvfp4_linear_fwd_noalloc(_ptr(X), _ptr(W), _ptr(out), M, N, K, _dtype_code(X.dtype),
                                          _dtype_code(out.dtype), _stream(stream))
     _ok(st, "nvfp4_linear_fwd_noalloc")
     return out
 
 
+def _bf16_like(name, t, ref):
+    _dense(name, t, shape=tuple(ref.shape), dtype=torch.bfloat16)
+
+
 def nvfp4_relu2_fwd(y, out=None, stream=None):
+    _dense("y", y, dtype=torch.bfloat16)
     out = out if out is not None else torch.empty_like(y)
+    _bf16_like("out", out, y)
+    _on_device(y, out)
     _ok(load().nvfp4_relu2_fwd(_ptr(y), _ptr(out), y.numel(), _stream(stream)), "nvfp4_relu2_fwd")
     return out
 
 
 def nvfp4_relu2_bwd(dh, y, out=None, stream=None):
+    _dense("y", y, dtype=torch.bfloat16)
+    _bf16_like("dh", dh, y)
     out = out if out is not None else torch.empty_like(y)
+    _bf16_like("out", out, y)
+    _on_device(dh, y, out)
     _ok(load().nvfp4_relu2_bwd(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _stream(stream)), "nvfp4_relu2_bwd")
     return out
 
 
+def _amax_buffer(t, device):
+    t = t if t is not None else torch.empty(4, dtype=torch.float32, device=device)
+    _scalar_out("amax output", t)
+    return t
+
+
 def nvfp4_relu2_fwd_amax(y, out=None, amax_out=None, ws=None, stream=None):
     """relu(y)^2 and max |output| (a 1-element float32 CUDA tensor); returns (out, amax_out)."""
+    _dense("y", y, dtype=torch.bfloat16)
     out = out if out is not None else torch.empty_like(y)
-    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    _bf16_like("out", out, y)
+    amax_out = _amax_buffer(amax_out, y.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), y.device)
-    _ok(load().nvfp4_relu2_fwd_amax(_ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), ws.numel(),
+    _on_device(y, out, amax_out, ws)
+    _ok(load().nvfp4_relu2_fwd_amax(_ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), _workspace(ws),
                                     _stream(stream)), "nvfp4_relu2_fwd_amax")
     return out, amax_out
 
 
 def nvfp4_relu2_bwd_amax(dh, y, out=None, amax_out=None, ws=None, stream=None):
     """dh * 2 relu(y) and max |output|; returns (out, amax_out)."""
+    _dense("y", y, dtype=torch.bfloat16)
+    _bf16_like("dh", dh, y)
     out = out if out is not None else torch.empty_like(y)
-    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
+    _bf16_like("out", out, y)
+    amax_out = _amax_buffer(amax_out, y.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), y.device)
-    _ok(load().nvfp4_relu2_bwd_amax(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws), ws.numel(),
-                                    _stream(stream)), "nvfp4_relu2_bwd_amax")
+    _on_device(dh, y, out, amax_out, ws)
+    _ok(load().nvfp4_relu2_bwd_amax(_ptr(dh), _ptr(y), _ptr(out), y.numel(), _ptr(amax_out), _ptr(ws),
+                                    _workspace(ws), _stream(stream)), "nvfp4_relu2_bwd_amax")
     return out, amax_out
 
 
 def nvfp4_relu2_fwd_amax_rht(y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
     """relu(y)^2 of a 2-D bf16 tensor plus max|out| and max|RHT(out)|; returns (out, amax, amax_rht)."""
+    _rows("y", y)
+    _dense("y", y, dtype=torch.bfloat16)
     R, Cc = y.shape
     out = out if out is not None else torch.empty_like(y)
-    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
-    amax_rht_out = amax_rht_out if amax_rht_out is not None else torch.empty(4, dtype=torch.float32,
-                                                                             device=y.device)
+    _bf16_like("out", out, y)
+    amax_out = _amax_buffer(amax_out, y.device)
+    amax_rht_out = _amax_buffer(amax_rht_out, y.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), y.device)
+    _on_device(y, out, amax_out, amax_rht_out, ws)
     _ok(load().nvfp4_relu2_fwd_amax_rht(_ptr(y), _ptr(out), R, Cc, seed, _ptr(amax_out), _ptr(amax_rht_out),
-                                        _ptr(ws), ws.numel(), _stream(stream)), "nvfp4_relu2_fwd_amax_rht")
+                                        _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_relu2_fwd_amax_rht")
     return out, amax_out, amax_rht_out
 
 
 def nvfp4_relu2_bwd_amax_rht(dh, y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
     """dh * 2 relu(y) of 2-D bf16 tensors plus max|out| and max|RHT(out)|; returns (out, amax, amax_rht)."""
+    _rows("y", y)
+    _dense("y", y, dtype=torch.bfloat16)
+    _bf16_like("dh", dh, y)
     R, Cc = y.shape
     out = out if out is not None else torch.empty_like(y)
-    amax_out = amax_out if amax_out is not None else torch.empty(4, dtype=torch.float32, device=y.device)
-    amax_rht_out = amax_rht_out if amax_rht_out is not None else torch.empty(4, dtype=torch.float32,
-                                                                             device=y.device)
+    _bf16_like("out", out, y)
+    amax_out = _amax_buffer(amax_out, y.device)
+    amax_rht_out = _amax_buffer(amax_rht_out, y.device)
     ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), y.device)
+    _on_device(dh, y, out, amax_out, amax_rht_out, ws)
     _ok(load().nvfp4_relu2_bwd_amax_rht(_ptr(dh), _ptr(y), _ptr(out), R, Cc, seed, _ptr(amax_out),
-                                        _ptr(amax_rht_out), _ptr(ws), ws.numel(), _stream(stream)),
+                                        _ptr(amax_rht_out), _ptr(ws), _workspace(ws), _stream(stream)),
         "nvfp4_relu2_bwd_amax_rht")
     return out, amax_out, amax_rht_out
 
 
 def nvfp4_check(ws, stream=None):
     """Synchronise and read/clear the workspace status word; raises on a device error."""
+    _on_device(ws)
     _ok(load().nvfp4_check(_ptr(ws), _stream(stream)), "nvfp4_check")
 
 
 def nvfp4_selftest_wait_timeout(ws, limit_ns, stream=None):
     """Launch the device-timeout self-test (its status is read by nvfp4_check)."""
-    _ok(load().nvfp4_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(limit_ns), _stream(stream)),
+    _on_device(ws)
+    _ok(load().nvfp4_selftest_wait_timeout(_ptr(ws), _workspace(ws), int(limit_ns), _stream(stream)),
         "nvfp4_selftest_wait_timeout")
 
 
