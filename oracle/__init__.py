@@ -64,6 +64,7 @@ def lib():
         L.oracle_mx_scale.restype = C.c_uint
         L.oracle_quantize_mx.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_int, u8p, u8p]
         L.oracle_quantize_mx.restype = C.c_int
+        L.oracle_gemm_mx.argtypes = [u8p, u8p, u8p, u8p, C.c_int64, C.c_int64, C.c_int64, f64p, f64p]
         L.oracle_quantize_rows.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64,
                                            C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_float,
                                            i64p, C.c_int64, u8p, u8p]
@@ -312,6 +313,22 @@ def quantize_mx(x, colwise=False):
                                 _p(scales, C.c_uint8)) != 0:
         raise ValueError("oracle_quantize_mx rejected the arguments")
     return codes, scales
+
+
+def gemm_mx(a, b):
+    """FP64 GEMM of two MXFP4 tensors a, b = (codes [rows x K/2], scales [rows x K/32]).
+
+    Returns (ref [M x N], abs [M x N]) with ref = A.B^T, abs = sum |a_k b_k|."""
+    ac, asc = (np.ascontiguousarray(t, dtype=np.uint8) for t in a[:2])
+    bc, bsc = (np.ascontiguousarray(t, dtype=np.uint8) for t in b[:2])
+    M, N, K = ac.shape[0], bc.shape[0], ac.shape[1] * 2
+    if bc.shape[1] * 2 != K or K % 32 or asc.shape != (M, K // 32) or bsc.shape != (N, K // 32):
+        raise ValueError("MXFP4 operands: codes [rows x K/2], scales [rows x K/32], one K (a multiple of 32)")
+    ref = np.zeros((M, N), np.float64)
+    ab = np.zeros((M, N), np.float64)
+    lib().oracle_gemm_mx(_p(ac, C.c_uint8), _p(asc, C.c_uint8), _p(bc, C.c_uint8), _p(bsc, C.c_uint8), M, N, K,
+                         _p(ref, C.c_double), _p(ab, C.c_double))
+    return ref, ab
 
 
 def dequantize_mx(codes, scales):

@@ -47,6 +47,9 @@
  *   mx (MXFP4)        pinned: E8M0 values, shared exponent on binade
  *                     boundaries, exact round trip of every E2M1 code at many
  *                     exponents, saturation, the RTN error bound
+ *   gemm_mx           pinned: closed form K*e2m1*e2m1*2^(xa+xb), one-hot
+ *                     indexing across 32-blocks, exact agreement with the
+ *                     NVFP4 gemm on scales both formats represent
  *   Readings (tensor-scale constant 2688, the R8 counter mapping, the sign
  *   word of the Hadamard diagonal, multiply-by-reciprocal) are fixed by this
  *   file, not by the pages: "parity unpinned" for those choices themselves.
@@ -506,6 +509,34 @@ void oracle_gemm_sampled(const uint8_t *a_codes, const uint8_t *a_scales, float 
     for (int64_t i = 0; i < count; ++i)
         oracle_dot(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, K, ms[i], ns[i],
                    &ref[i], &absref[i]);
+}
+
+/* MXFP4 operands [AIS "Architektura NVFP4 kontra ograniczenia ..."]: the
+ * same binary64 dot product with E8M0 block scales over blocks of 32 and no
+ * tensor scale.  Codes packed as for NVFP4, scales plain [rows x K/32]. */
+static double deq_mx(const uint8_t *codes_row, const uint8_t *scales_row, int64_t k)
+{
+    uint8_t byte = codes_row[k >> 1];
+    unsigned q = (k & 1) ? (byte >> 4) : (byte & 0xFu);
+    return oracle_e2m1_value(q) * oracle_e8m0_value(scales_row[k >> 5]);
+}
+
+void oracle_gemm_mx(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *b_codes,
+                    const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, double *ref, double *absref)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t *ac = a_codes + m * (K / 2), *as = a_scales + m * (K / 32);
+            const uint8_t *bc = b_codes + n * (K / 2), *bs = b_scales + n * (K / 32);
+            double s = 0.0, sa = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = deq_mx(ac, as, k) * deq_mx(bc, bs, k);
+                s += p;
+                sa += fabs(p);
+            }
+            ref[m * N + n] = s;
+            absref[m * N + n] = sa;
+        }
 }
 
 /* ------------------------------------------------------------------------ */

@@ -119,3 +119,90 @@ def test_colwise_is_rowwise_of_the_transpose():
     assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
     with pytest.raises(ValueError):
         oracle.quantize_mx(np.zeros((48, 64), np.float32), colwise=True)   # R % 32 != 0
+
+
+# ---------------------------------------------------------------- MXFP4 GEMM
+def _pack_rows(codes):
+    codes = np.asarray(codes, np.uint8)
+    return codes[:, 0::2] | (codes[:, 1::2] << 4)
+
+
+def test_gemm_mx_closed_form():
+    """Every element of a row holds one code c and every block the row's exponent x:
+    C[m, n] = K * e2m1(c_m) * e2m1(c_n) * 2^(x_m + x_n) exactly."""
+    rng = np.random.default_rng(31)
+    M, N, K = 5, 7, 96
+    ca, cb = rng.integers(0, 16, M), rng.integers(0, 16, N)
+    xa, xb = rng.integers(-20, 21, M), rng.integers(-20, 21, N)
+    a = (_pack_rows(np.repeat(ca[:, None], K, 1)), np.repeat((xa + 127)[:, None], K // 32, 1).astype(np.uint8))
+    b = (_pack_rows(np.repeat(cb[:, None], K, 1)), np.repeat((xb + 127)[:, None], K // 32, 1).astype(np.uint8))
+    ref, ab = oracle.gemm_mx(a, b)
+    val = lambda c: (-1.0 if c & 8 else 1.0) * E2M1[c & 7]  # noqa: E731
+    want = np.array([[K * val(ca[m]) * val(cb[n]) * 2.0 ** (xa[m] + xb[n]) for n in range(N)] for m in range(M)])
+    assert np.array_equal(ref, want)
+    assert np.array_equal(ab, np.abs(want))
+
+
+def test_gemm_mx_one_hot_indexing():
+    """One nonzero per row at a known k, each 32-block with its own exponent: the product
+    is nonzero only where the positions meet, with both blocks' scales -- this pins
+    the nibble order and the block index k // 32."""
+    rng = np.random.default_rng(32)
+    K, R = 128, 12
+    pos_a, pos_b = rng.integers(0, K, R), rng.integers(0, K, R)
+    pos_b[:4] = pos_a[:4]
+    ea, eb = rng.integers(100, 150, (R, K // 32)), rng.integers(100, 150, (R, K // 32))
+    codes_a, codes_b = np.zeros((R, K), np.uint8), np.zeros((R, K), np.uint8)
+    codes_a[np.arange(R), pos_a] = 5   # 3.0
+    codes_b[np.arange(R), pos_b] = 11  # -1.5
+    ref, _ = oracle.gemm_mx((_pack_rows(codes_a), ea.astype(np.uint8)), (_pack_rows(codes_b), eb.astype(np.uint8)))
+    for m in range(R):
+        for n in range(R):
+            k = pos_a[m]
+            want = 3.0 * -1.5 * 2.0 ** (int(ea[m, k // 32]) - 127 + int(eb[n, k // 32]) - 127) if k == pos_b[n] else 0.0
+            assert ref[m, n] == want, (m, n)
+
+
+def _e4m3_code_of(v):
+    return next(c for c in range(127) if oracle.e4m3_value(c) == v)
+
+
+def test_gemm_mx_equals_nvfp4_gemm_on_shared_scales():
+    """An MXFP4 tensor whose block exponents are also E4M3 values is the NVFP4 tensor
+    with that scale on both 16-halves of each 32-block and tensor scale 1: the two
+    oracles' FP64 GEMMs (independent scale decoders and block sizes) agree exactly."""
+    rng = np.random.default_rng(33)
+    M, N, K = 9, 11, 160
+    def operand(rows):
+        codes = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+        x = rng.integers(-9, 9, (rows, K // 32))                  # 2^x is an E4M3 value for x in [-9, 8]
+        e8 = (x + 127).astype(np.uint8)
+        e4 = np.array([[_e4m3_code_of(2.0 ** int(v)) for v in row] for row in x], np.uint8)
+        return (codes, e8), (codes, np.repeat(e4, 2, axis=1), np.float32(1.0))
+    (amx, anv), (bmx, bnv) = operand(M), operand(N)
+    ref_mx, ab_mx = oracle.gemm_mx(amx, bmx)
+    ref_nv, ab_nv = oracle.gemm(anv, bnv)
+    assert np.array_equal(ref_mx, ref_nv)
+    assert np.array_equal(ab_mx, ab_nv)
+
+
+def test_gemm_mx_of_quantised_operands_tracks_the_product():
+    """gemm_mx(quantize_mx(X), quantize_mx(W)) approximates X W^T, and less closely
+    than the NVFP4 path on the same data (the pages' point about finer scaling)."""
+    rng = np.random.default_rng(34)
+    X = rng.standard_normal((64, 512)).astype(np.float32)
+    W = rng.standard_normal((48, 512)).astype(np.float32)
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    ref_mx, _ = oracle.gemm_mx(oracle.quantize_mx(X), oracle.quantize_mx(W))
+    ref_nv, _ = oracle.gemm(oracle.quantize(X)[:3], oracle.quantize(W)[:3])
+    err_mx = np.linalg.norm(ref_mx - exact) / np.linalg.norm(exact)
+    err_nv = np.linalg.norm(ref_nv - exact) / np.linalg.norm(exact)
+    assert err_mx < 0.25 and err_nv < err_mx, (err_mx, err_nv)
+
+
+def test_gemm_mx_rejects_mismatched_operands():
+    c, s = np.zeros((4, 16), np.uint8), np.zeros((4, 1), np.uint8)
+    with pytest.raises(ValueError):
+        oracle.gemm_mx((c, s), (np.zeros((4, 32), np.uint8), np.zeros((4, 2), np.uint8)))
+    with pytest.raises(ValueError):
+        oracle.gemm_mx((c, np.zeros((4, 2), np.uint8)), (c, s))
