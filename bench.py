@@ -327,7 +327,7 @@ def oracle_sample(budget_s=12.0):
     import oracle
     rng = np.random.default_rng(0)
     t_all = time.perf_counter()
-    # quantiser: per-element cost of each mode on a 256 x 5120 bf16 slice (amax + quantise)
+    # quantiser: per-element cost of each mode on a 2048 x 5120 bf16 slice (amax + quantise)
     x = W.bf16_bits(W.normal(rng, (2048, 5120)))
     per_elem = {}
     for mode in [(False, False, False), (True, False, False), (True, True, True), (True, False, True)]:
