@@ -180,6 +180,9 @@ NVFP4_API nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int
  * multiple of 16, and M, N, K < 2^31.  M or N == 0: nothing is done.
  * K == 0: C is zero-filled.
  * workspace: >= 256 bytes (status word).
+ * Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_SHAPE, NVFP4_ERR_ALIGNMENT,
+ * NVFP4_ERR_WORKSPACE, NVFP4_ERR_UNSUPPORTED_DEVICE, NVFP4_ERR_CUDA; a device
+ * timeout is recorded in the workspace status word (nvfp4_check).
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
                         int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
@@ -191,7 +194,10 @@ NVFP4_API size_t nvfp4_linear_workspace_size(int64_t M, int64_t N, int64_t K);
  * nvfp4_linear_fwd -- Fprop of Y = X . W^T: X [M x K], W [N x K] (dtype,
  * row-major, contiguous) -> Y [M x N] (y_dtype, contiguous).  Both operands
  * are quantised rowwise with round-to-nearest-even, then nvfp4_gemm.
- * Requires K % 64 == 0; quantised operands live in the workspace.
+ * Requires K % 64 == 0; quantised operands live in the workspace
+ * (>= nvfp4_linear_workspace_size(M, N, K) bytes, 16-byte aligned, zeroed
+ * status word).  M or N == 0: nothing is done.
+ * Errors: as nvfp4_quantize and nvfp4_gemm.
  */
 NVFP4_API nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
                               nvfp4_dtype dtype, nvfp4_dtype y_dtype,
@@ -206,7 +212,9 @@ NVFP4_API nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, i
  * operands only (aisight.pl, section "Technologie stabilizujace proces
  * treningowy"); both Wgrad operands use the same signs, from `seed`, which
  * also keys the SR draws.  dY's two operands come from one read of dY
- * (nvfp4_quantize_dual).  Requires M % 64 == 0, N % 64 == 0, K % 64 == 0.
+ * (nvfp4_quantize_dual).  Requires M, N, K > 0 and multiples of 64, and
+ * M, N <= 65535 * 256 (the colwise quantisations' limit); workspace as for
+ * nvfp4_linear_fwd.  Errors: as nvfp4_quantize and nvfp4_gemm.
  */
 NVFP4_API nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const void *W, void *dX, float *dW,
                               int64_t M, int64_t N, int64_t K, nvfp4_dtype dtype,
