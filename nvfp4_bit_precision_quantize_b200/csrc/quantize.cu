@@ -1,11 +1,14 @@
 // quantize.cu -- NVFP4 quantisation kernels for sm_100a.
 //
-// Two passes over the input, both HBM-bound:
-//   pass 1 (amax_*): tensor amax (after the random Hadamard transform when it
-//     is on), written as one partial per CTA -- no atomics, no zeroing;
+// Two passes over the input:
+//   pass 1 (amax_*, HBM-bound): tensor amax (after the random Hadamard
+//     transform when it is on), written as one partial per CTA -- no atomics,
+//     no zeroing;
 //   pass 2 (quantize_*): every CTA reduces the partials to the same amax,
 //     derives the FP32 tensor scale, and turns its tile into packed E2M1 codes
 //     plus E4M3 block scales laid out in the tensor cores' 128x4 scale atoms.
+//     HBM-bound in design; with the Hadamard transform and stochastic rounding
+//     (Philox per 8 elements) the colwise variant is bound by ALU issue instead.
 // Format: aisight.pl, "Koniec marnowania mocy ...", section "Architektura
 // NVFP4 kontra ograniczenia mikroskalowania" (block 16, E4M3 block scale, FP32
 // tensor scale).  Hadamard transform and stochastic rounding on the Wgrad
