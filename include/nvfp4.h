@@ -187,17 +187,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
                         int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
 
-/* Workspace bytes for nvfp4_linear_fwd / nvfp4_linear_bwd at these sizes. */
+/* Workspace bytes at these sizes: nvfp4_linear_workspace_size serves both
+ * nvfp4_linear_fwd and nvfp4_linear_bwd (the larger of the two footprints);
+ * nvfp4_linear_fwd_workspace_size is what nvfp4_linear_fwd alone needs (the
+ * status word, amax partials, tensor scales and the two rowwise operands).
+ * Both return 0 for negative sizes. */
 NVFP4_API size_t nvfp4_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+NVFP4_API size_t nvfp4_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
  * nvfp4_linear_fwd -- Fprop of Y = X . W^T: X [M x K], W [N x K] (dtype,
- * row-major, contiguous) -> Y [M x N] (y_dtype, contiguous).  Both operands
- * are quantised rowwise with round-to-nearest-even, then nvfp4_gemm.
+ * row-major, contiguous) -> Y [M x N] (y_dtype, contiguous).  The forward
+ * GEMM of a layer trained in 4 bits, the step hyper.ai ("NVIDIA
+ * revolutioniert KI-Praetrainingsgeschwindigkeit mit 4-Bit-Genauigkeit")
+ * credits with the GEMM speed-up, on operands in the format of aisight.pl,
+ * section "Architektura NVFP4 kontra ograniczenia mikroskalowania" (blocks of
+ * 16, E4M3 block scale, FP32 tensor scale).  The Hadamard transform and
+ * stochastic rounding are for the weight gradients only (same page, section
+ * "Technologie stabilizujace proces treningowy"), so both operands are
+ * quantised rowwise with round-to-nearest-even (nvfp4_quantize, two passes
+ * each), then multiplied by nvfp4_gemm.
  * Requires K % 64 == 0; quantised operands live in the workspace
- * (>= nvfp4_linear_workspace_size(M, N, K) bytes, 16-byte aligned, zeroed
- * status word).  M or N == 0: nothing is done.
- * Errors: as nvfp4_quantize and nvfp4_gemm.
+ * (>= nvfp4_linear_fwd_workspace_size(M, N, K) bytes, 16-byte aligned,
+ * device memory, caller-owned, zeroed status word).  M or N == 0: nothing is
+ * done.  Errors: as nvfp4_quantize and nvfp4_gemm, checked before any launch.
  */
 NVFP4_API nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
                               nvfp4_dtype dtype, nvfp4_dtype y_dtype,
@@ -231,13 +244,15 @@ NVFP4_API nvfp4_status nvfp4_linear_bwd(const void *dY, const void *X, const voi
  * the scratch (status word, amax partials, both quantised operands) is one
  * fixed device buffer of NVFP4_NOALLOC_SCRATCH_BYTES inside the library, which
  * every GPU that loads the library holds until the process exits.  Calls
- * whose nvfp4_linear_workspace_size(M, N, K) exceeds it return
+ * whose nvfp4_linear_fwd_workspace_size(M, N, K) exceeds it return
  * NVFP4_ERR_WORKSPACE and launch nothing.  The first call on a device looks
  * the buffer's address up (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  The call allocates and
- * frees nothing.  All calls share the one buffer and each starts by zeroing
- * its status word: calls that overlap on the GPU (other streams, other host
- * threads) race on it and must be serialised by the caller.  A device-side
+ * frees nothing.  All calls share the one buffer and each call that passes
+ * its checks starts by zeroing the status word (a refused call touches
+ * neither the buffer nor the stream): calls that overlap on the GPU (other
+ * streams, other host threads) race on it and must be serialised by the
+ * caller.  A device-side
  * timeout is recorded only in that shared buffer, which no public call reads.
  */
 #define NVFP4_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -36,7 +36,7 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
-           "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht")
+           "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size")
 
 
 class CTensor(C.Structure):
@@ -70,6 +70,7 @@ def load():
         "nvfp4_quantize": (i32, [vp, i32, i64, i64, i64, i32, i32, i32, u64, vp, tp, vp, sz, vp]),
         "nvfp4_gemm": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
         "nvfp4_linear_workspace_size": (sz, [i64, i64, i64]),
+        "nvfp4_linear_fwd_workspace_size": (sz, [i64, i64, i64]),
         "nvfp4_linear_fwd": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]),
         "nvfp4_linear_bwd": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, u64, vp, sz, vp]),
         "nvfp4_relu2_fwd": (i32, [vp, vp, i64, vp]),
@@ -218,6 +219,10 @@ def nvfp4_linear_workspace_size(M, N, K):
     return load().nvfp4_linear_workspace_size(M, N, K)
 
 
+def nvfp4_linear_fwd_workspace_size(M, N, K):
+    return load().nvfp4_linear_fwd_workspace_size(M, N, K)
+
+
 def workspace(nbytes, device=None):
     """A zeroed workspace (its status word must start at zero)."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
@@ -329,7 +334,7 @@ def _linear_operands(X, W):
 def nvfp4_linear_fwd(X, W, y_dtype=torch.bfloat16, out=None, ws=None, stream=None):
     M, N, K = _linear_operands(X, W)
     out = out if out is not None else torch.empty((M, N), dtype=y_dtype, device=X.device)
-    ws = ws if ws is not None else workspace(nvfp4_linear_workspace_size(M, N, K), X.device)
+    ws = ws if ws is not None else workspace(nvfp4_linear_fwd_workspace_size(M, N, K), X.device)
     _dense("out", out, shape=(M, N))
     _on_device(X, W, out, ws)
     st = load().nvfp4_linear_fwd(_ptr(X), _ptr(W), _ptr(out), M, N, K, _dtype_code(X.dtype),

@@ -239,6 +239,37 @@ nvfp4_status dual_impl(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, i
 
 }  // namespace
 
+namespace nvfp4 {
+
+size_t linear_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 0 || K < 0) return 0;
+    return fwd_bytes(M, N, K);
+}
+
+// Every host-side check nvfp4_linear_fwd makes before it launches anything,
+// device check included; M or N == 0 passes (nothing to do).
+nvfp4_status linear_fwd_validate(const void *X, const void *W, const void *Y, int64_t M, int64_t N, int64_t K,
+                                 nvfp4_dtype dtype, nvfp4_dtype y_dtype, const void *workspace, size_t ws_bytes) {
+    if (!valid_dtype(dtype) || !valid_dtype(y_dtype)) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || K % 64 != 0) return NVFP4_ERR_SHAPE;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!X || !W || !Y) return NVFP4_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < fwd_bytes(M, N, K)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    uint8_t *ws = static_cast<uint8_t *>(const_cast<void *>(workspace));
+    float *ts = reinterpret_cast<float *>(ws + kScalarsOff);
+    Carver cv{ws, kBuffersOff};
+    const nvfp4_tensor xq = cv.take(M, K, ts + 0), wq = cv.take(N, K, ts + 1);
+    nvfp4_status st;
+    if ((st = validate_quantize(X, dtype, M, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, nullptr, &xq, ws, ws_bytes)) ||
+        (st = validate_quantize(W, dtype, N, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, nullptr, &wq, ws, ws_bytes)) ||
+        (st = validate_gemm(&xq, &wq, Y, y_dtype, N, ws, ws_bytes)))
+        return st;
+    return check_device();
+}
+
+}  // namespace nvfp4
+
 extern "C" {
 
 size_t nvfp4_codes_bytes(int64_t rows, int64_t k) {
@@ -258,6 +289,10 @@ size_t nvfp4_quantize_workspace_size(void) { return kQuantizeWorkspace; }
 size_t nvfp4_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M < 0 || N < 0 || K < 0) return 0;
     return std::max(fwd_bytes(M, N, K), bwd_bytes(M, N, K));
+}
+
+size_t nvfp4_linear_fwd_workspace_size(int64_t M, int64_t N, int64_t K) {
+    return nvfp4::linear_fwd_workspace_bytes(M, N, K);
 }
 
 nvfp4_status nvfp4_quantize(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int orientation,
@@ -335,22 +370,13 @@ nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, 
                               nvfp4_dtype dtype, nvfp4_dtype y_dtype, void *workspace, size_t ws_bytes,
                               cudaStream_t stream) {
     Call call(__func__);
-    if (!valid_dtype(dtype) || !valid_dtype(y_dtype)) return NVFP4_ERR_INVALID_ARG;
-    if (M < 0 || N < 0 || K < 0 || K % 64 != 0) return NVFP4_ERR_SHAPE;
+    nvfp4_status st = nvfp4::linear_fwd_validate(X, W, Y, M, N, K, dtype, y_dtype, workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
     if (M == 0 || N == 0) return call.done(NVFP4_OK);
-    if (!X || !W || !Y) return NVFP4_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < nvfp4_linear_workspace_size(M, N, K)) return NVFP4_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *ts = reinterpret_cast<float *>(ws + kScalarsOff);
     Carver cv{ws, kBuffersOff};
     const nvfp4_tensor xq = cv.take(M, K, ts + 0), wq = cv.take(N, K, ts + 1);
-    nvfp4_status st;
-    if ((st = validate_quantize(X, dtype, M, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, nullptr, &xq, ws, ws_bytes)) ||
-        (st = validate_quantize(W, dtype, N, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, nullptr, &wq, ws, ws_bytes)) ||
-        (st = validate_gemm(&xq, &wq, Y, y_dtype, N, ws, ws_bytes)))
-        return st;
-    if ((st = check_device()) != NVFP4_OK) return st;
     if ((st = quantize_impl(X, dtype, M, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, 0, nullptr, &xq, ws, stream,
                             &call.launches)) ||
         (st = quantize_impl(W, dtype, N, K, K, NVFP4_ROWWISE, NVFP4_RTN, 0, 0, nullptr, &wq, ws, stream,

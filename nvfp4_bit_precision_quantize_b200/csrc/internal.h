@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "nvfp4.h"
+
 namespace nvfp4 {
 
 constexpr int kMaxPartials = 1024;          // per-CTA amax partials in a quantize workspace
@@ -77,5 +79,12 @@ cudaError_t launch_relu2_amax_rht(const void *dh, const void *y, void *out, int6
                                   int *launches);
 
 int num_sms();  // SM count of the current device (cached)
+
+// Scratch bytes nvfp4_linear_fwd needs (both rowwise operands after the
+// status word, amax partials and tensor scales), and every host-side check it
+// makes before launching, device check included (M or N == 0 passes).
+size_t linear_fwd_workspace_bytes(int64_t M, int64_t N, int64_t K);
+nvfp4_status linear_fwd_validate(const void *X, const void *W, const void *Y, int64_t M, int64_t N, int64_t K,
+                                 nvfp4_dtype dtype, nvfp4_dtype y_dtype, const void *workspace, size_t ws_bytes);
 
 }  // namespace nvfp4

@@ -47,11 +47,16 @@ extern "C" nvfp4_status nvfp4_linear_fwd_noalloc(const void *X, const void *W, v
                                                  int64_t K, nvfp4_dtype dtype, nvfp4_dtype y_dtype,
                                                  cudaStream_t stream) {
     if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_SHAPE;
-    // Problems whose scratch exceeds the fixed buffer are refused before anything runs.
-    if (nvfp4_linear_workspace_size(M, N, K) > kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;
+    // Problems whose scratch (the forward operands only) exceeds the fixed
+    // buffer are refused before anything runs.
+    if (nvfp4::linear_fwd_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;
     if (M == 0 || N == 0) return nvfp4_linear_fwd(X, W, Y, M, N, K, dtype, y_dtype, nullptr, 0, stream);
     uint8_t *scratch = nullptr;
     nvfp4_status st = scratch_address(&scratch);
+    if (st != NVFP4_OK) return st;
+    // Every check nvfp4_linear_fwd makes runs first, so a refused call touches
+    // neither the shared buffer nor the stream.
+    st = nvfp4::linear_fwd_validate(X, W, Y, M, N, K, dtype, y_dtype, scratch, kNoAllocScratchBytes);
     if (st != NVFP4_OK) return st;
     // The device status word must start at zero; the rest is overwritten before it is read.
     if (cudaMemsetAsync(scratch, 0, nvfp4::kStatusBytes, stream) != cudaSuccess) return NVFP4_ERR_CUDA;

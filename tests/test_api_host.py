@@ -43,6 +43,13 @@ def test_sizes(lib):
         assert lib.nvfp4_scales_bytes(rows, k) == layout.scales_bytes(rows, k)
     assert lib.nvfp4_quantize_workspace_size() >= 256 + 4 * 1024
     assert lib.nvfp4_linear_workspace_size(8192, 20480, 5120) > 0.5625 * 8192 * 20480 * 2
+    # forward footprint: the rowwise X [M x K] and W [N x K] operands, plus the fixed header
+    for M, N, K in [(8192, 20480, 5120), (256, 4096, 64), (128, 128, 128)]:
+        fwd = lib.nvfp4_linear_fwd_workspace_size(M, N, K)
+        ops = sum(lib.nvfp4_codes_bytes(r, K) + lib.nvfp4_scales_bytes(r, K) for r in (M, N))
+        assert ops <= fwd <= ops + 16384
+        assert fwd <= lib.nvfp4_linear_workspace_size(M, N, K)
+    assert lib.nvfp4_linear_fwd_workspace_size(-1, 1, 64) == 0
 
 
 def test_status_strings(lib):
@@ -111,7 +118,9 @@ def test_linear_rejections(lib):
     p = C.c_void_p
     assert lib.nvfp4_linear_fwd(p(0x1000), p(0x2000), p(0x3000), 128, 128, 96, 1, 1, p(0x4000), ws, None) \
         == E.NVFP4_ERR_SHAPE
-    assert lib.nvfp4_linear_fwd(p(0x1000), p(0x2000), p(0x3000), 128, 128, 128, 1, 1, p(0x4000), ws - 1,
+    wsf = lib.nvfp4_linear_fwd_workspace_size(128, 128, 128)
+    assert wsf < ws                                                   # the forward pass needs 2 of the 4 operands
+    assert lib.nvfp4_linear_fwd(p(0x1000), p(0x2000), p(0x3000), 128, 128, 128, 1, 1, p(0x4000), wsf - 1,
                                 None) == E.NVFP4_ERR_WORKSPACE
     assert lib.nvfp4_linear_fwd(None, p(0x2000), p(0x3000), 128, 128, 128, 1, 1, p(0x4000), ws, None) \
         == E.NVFP4_ERR_INVALID_ARG
