@@ -27,6 +27,33 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     return c;
 }
 
+// The same generator with its ten round keys computed once (the key schedule
+// depends only on the seed), and each 32x32 -> 64-bit product taken whole.
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+    PhiloxKeys k;
+    uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        k.k0[round] = a;
+        k.k1[round] = b;
+        a += 0x9E3779B9u;
+        b += 0xBB67AE85u;
+    }
+    return k;
+}
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys &k) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c.x, p1 = (uint64_t)0xCD9E8D57u * c.z;
+        c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k.k0[round], (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k.k1[round],
+                       (uint32_t)p0);
+    }
+    return c;
+}
+
 // 16 sign bits of the Hadamard diagonal: word 0 of the block at counter (0,0,1,0).
 __device__ __forceinline__ uint32_t rht_sign_bits(uint64_t seed) {
     return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), (uint32_t)seed, (uint32_t)(seed >> 32)).x & 0xFFFFu;
@@ -64,19 +91,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
 // ---------------------------------------------------------------------------
 // Format conversions (hardware cvt, round-to-nearest-even, satfinite)
 // ---------------------------------------------------------------------------
-// E4M3 code of t >= 0 (values above 448 saturate to 448 = 0x7E).
-__device__ __forceinline__ uint32_t e4m3_code(float t) {
-    uint16_t out;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(t));
-    return out & 0xFFu;
-}
-
-// Exact value of an unsigned E4M3 code (0x7F never occurs here).
-__device__ __forceinline__ float e4m3_value(uint32_t c) {
-    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
-}
-
 // Four E2M1 codes from four floats (element 0 in the lowest nibble) -> 16 bits.
 __device__ __forceinline__ uint32_t e2m1x4(float a, float b, float c, float d) {
     uint16_t out;
@@ -113,37 +127,101 @@ __device__ __forceinline__ uint32_t e2m1x8(const float *v) {
 // 0.5-grid on the first mantissa bit; the sum is rounded UP to binary32, which
 // keeps the comparison with the 2^-17-spaced threshold exact (a threshold t on
 // the binary32 grid has x > t iff roundup(x) > t), and 1 is subtracted again
-// (exact).  Values at or above 6 land on 6 or above and are clamped to 6.
-// Returns the exact E2M1 value (sign of r kept), to be encoded by e2m1x*.
-__device__ __forceinline__ float sr_e2m1_value(float r, uint32_t rnd16) {
-    const float a = fabsf(r);
+// (exact).  Magnitudes are first clamped to 7: everything from 6 up lands on 6
+// or 8, which the saturating E2M1 conversion turns into 6.
+// `carry` = (2^16 - 1 - rnd16) * 2^6 + 63 (sr_carry_lo / sr_carry_hi below).
+// Returns the E2M1 value (or 8 for 6), sign of r kept, for e2m1x*.
+__device__ __forceinline__ float sr_e2m1_value(float r, uint32_t carry) {
+    const float a = fminf(fabsf(r), 7.0f);
     const float base = a < 1.0f ? 1.0f : 0.0f;
     const float t = __fadd_ru(a, base);
-    const uint32_t carry_in = ((~rnd16 & 0xFFFFu) << 6) | 63u;
-    const float up = __uint_as_float((__float_as_uint(t) + carry_in) & 0xFFC00000u);
-    const float mag = fminf(__fsub_rn(up, base), 6.0f);
-    return copysignf(mag, r);
+    const float up = __uint_as_float((__float_as_uint(t) + carry) & 0xFFC00000u);
+    return copysignf(__fsub_rn(up, base), r);
 }
+// carry of the low / high 16-bit draw of a Philox output word
+__device__ __forceinline__ uint32_t sr_carry_lo(uint32_t w) { return ((~w & 0xFFFFu) << 6) | 63u; }
+__device__ __forceinline__ uint32_t sr_carry_hi(uint32_t w) { return ((~w >> 16) << 6) | 63u; }
 
 // ---------------------------------------------------------------------------
-// Per-block scale computation shared by the quantisers:
-//   sb = E4M3(amax_b / 6 / s_t), dec = e4m3(sb) * s_t, inv = 1 / dec.
+// Per-block scale:  sb = E4M3(RN(RN(amax_b / 6) / s_t)),  dec = e4m3(sb) * s_t,
+// inv = RN(1 / dec); a block with sb = 0 (or dec = 0, or inv not finite) has
+// every code +0.
+//
+// The two divisions use Markstein's correction step (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Develop. 34(1), 1990): with rb = RN(1/b),
+// q0 = RN(a * rb), the residual r = a - q0 * b is exact in one FMA and
+// RN(q0 + r * rb) is the correctly rounded a / b, provided nothing underflows
+// or overflows.  For b = 6 this holds for every finite a >= 2^-125 (checked on
+// the CPU against IEEE division for every binary32 value).  For b = s_t it
+// holds whenever s_t lies in [2^-80, 2^100] and the quotient in
+// [2^-12, 2^10]; outside that window the code is decided anyway: quotients
+// below 2^-11 give sb = 0 whether or not they are correctly rounded, and a
+// numerator clamped to s_t * 2^10 gives 1024, which saturates to 448 like
+// every true quotient above it.  Tensor scales outside [2^-80, 2^100] (a
+// uniform condition) take IEEE divisions instead.
+// inv only depends on sb, so each CTA tabulates it once (scale_table_init)
+// with an IEEE division per code.
 // ---------------------------------------------------------------------------
-struct BlockScale {
-    uint32_t sb;
-    float inv;
-    bool zero;  // every code of the block is +0
+struct ScaleCtx {
+    float s_t;     // tensor scale
+    float rcp_st;  // RN(1 / s_t)
+    float st_hi;   // s_t * 2^10 (numerator clamp)
+    bool fast;     // s_t in [2^-80, 2^100]
 };
 
-__device__ __forceinline__ BlockScale block_scale(float amax_b, float s_t) {
-    BlockScale s;
-    float t = __fdiv_rn(amax_b, 6.0f);
-    t = __fdiv_rn(t, s_t);
-    s.sb = e4m3_code(t);
-    const float dec = __fmul_rn(e4m3_value(s.sb), s_t);
-    s.inv = __fdiv_rn(1.0f, dec);
-    s.zero = (s.sb == 0u) || (dec == 0.0f) || !isfinite(s.inv);
-    return s;
+__device__ __forceinline__ ScaleCtx scale_ctx(float s_t) {
+    ScaleCtx c;
+    c.s_t = s_t;
+    c.fast = s_t >= 0x1p-80f && s_t <= 0x1p+100f;
+    c.rcp_st = c.fast ? __fdiv_rn(1.0f, s_t) : 0.0f;
+    c.st_hi = s_t * 1024.0f;
+    return c;
+}
+
+__device__ __forceinline__ float div_markstein(float a, float b, float rb) {
+    const float q0 = __fmul_rn(a, rb);
+    const float r = __fmaf_rn(-q0, b, a);
+    return __fmaf_rn(r, rb, q0);
+}
+
+// E4M3 code of t >= 0 (values above 448 saturate to 448 = 0x7E).
+__device__ __forceinline__ uint32_t e4m3_code(float t) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(t));
+    return out & 0xFFu;
+}
+
+__device__ __forceinline__ uint32_t block_scale_code(float amax_b, const ScaleCtx &c) {
+    float t2;
+    if (c.fast) {
+        const float t = fminf(div_markstein(amax_b, 6.0f, 0x1.555556p-3f), c.st_hi);  // RN(1/6)
+        t2 = div_markstein(t, c.s_t, c.rcp_st);
+    } else {
+        t2 = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), c.s_t);
+    }
+    return e4m3_code(t2);
+}
+
+// Exact value of an unsigned E4M3 code (0x7F never occurs here).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+}
+
+// inv for every code (0 where the block's codes are all +0), and with `quarter`
+// also inv / 4 (exact when the context is fast), for the Hadamard-transformed
+// blocks whose 1/4 normalisation is folded into the element scale.  Threads
+// 0..127 fill one entry each; the caller synchronises before use.
+__device__ __forceinline__ void scale_table_init(float *inv_tab, float *inv4_tab, float s_t) {
+    if (threadIdx.x < 128) {
+        const uint32_t sb = threadIdx.x;
+        const float dec = __fmul_rn(e4m3_value(sb), s_t);
+        float inv = __fdiv_rn(1.0f, dec);
+        if (sb == 0u || sb == 127u || dec == 0.0f || !isfinite(inv)) inv = 0.0f;
+        inv_tab[sb] = inv;
+        if (inv4_tab) inv4_tab[sb] = __fmul_rn(inv, 0.25f);
+    }
 }
 
 __device__ __forceinline__ float tensor_scale_from_amax(float amax) {
@@ -161,9 +239,8 @@ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t b, int64_t KB
 // 16-point random Hadamard transform in registers: sign flips (xor of the sign
 // bit), the fixed-order butterfly over strides 1, 2, 4, 8, then a 1/4 scale.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void rht16(float *v, uint32_t signs) {
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(__float_as_uint(v[j]) ^ (((signs >> j) & 1u) << 31));
+// The fixed-order butterfly alone (strides 1, 2, 4, 8), unnormalised: z = H16 v.
+__device__ __forceinline__ void fwht16(float *v) {
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
@@ -174,6 +251,11 @@ __device__ __forceinline__ void rht16(float *v, uint32_t signs) {
             v[i + h] = __fsub_rn(a, b);
         }
     }
+}
+__device__ __forceinline__ void rht16(float *v, uint32_t signs) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(__float_as_uint(v[j]) ^ (((signs >> j) & 1u) << 31));
+    fwht16(v);
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
 }

@@ -23,6 +23,16 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// xor of a 16-byte row chunk with the sign-bit mask of Hadamard input row i
+// (bit i of the sign word set: every element of the chunk changes sign).
+template <typename T>
+__device__ __forceinline__ uint32_t sign_mask(uint32_t signs, int i) {
+    return ((signs >> i) & 1u) ? (sizeof(T) == 2 ? 0x80008000u : 0x80000000u) : 0u;
+}
+__device__ __forceinline__ uint4 xor4(const uint4 &a, uint32_t f) {
+    return make_uint4(a.x ^ f, a.y ^ f, a.z ^ f, a.w ^ f);
+}
+
 // ---------------------------------------------------------------------------
 // Pass 1a: max |x| over an [R x C] tensor (any orientation, no transform).
 // ---------------------------------------------------------------------------
@@ -99,6 +109,8 @@ __global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict_
 #pragma unroll
         for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
 #pragma unroll
+        for (int i = 0; i < 16; ++i) raw[i] = xor4(raw[i], sign_mask<T>(signs, i));
+#pragma unroll
         for (int j = 0; j < N; ++j) {
             float v[16];
 #pragma unroll
@@ -107,11 +119,12 @@ __global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict_
                 Vec<T>::unpack(raw[i], t);
                 v[i] = t[j];
             }
-            rht16(v, signs);
+            fwht16(v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
         }
     }
+    m = __fmul_rn(m, 0.25f);  // max |z / 4| = RN(max |z| / 4)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
@@ -146,6 +159,8 @@ __global__ void __launch_bounds__(kThreads) amax_dual_kernel(const T *__restrict
 #pragma unroll
         for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
 #pragma unroll
+        for (int i = 0; i < 16; ++i) raw[i] = xor4(raw[i], sign_mask<T>(signs, i));
+#pragma unroll
         for (int j = 0; j < N; ++j) {
             float v[16];
 #pragma unroll
@@ -153,13 +168,14 @@ __global__ void __launch_bounds__(kThreads) amax_dual_kernel(const T *__restrict
                 float t[N];
                 Vec<T>::unpack(raw[i], t);
                 v[i] = t[j];
-                m0 = fmaxf(m0, fabsf(v[i]));
+                m0 = fmaxf(m0, fabsf(v[i]));  // the sign flips do not change |v|
             }
-            rht16(v, signs);
+            fwht16(v);
 #pragma unroll
             for (int i = 0; i < 16; ++i) m1 = fmaxf(m1, fabsf(v[i]));
         }
     }
+    m1 = __fmul_rn(m1, 0.25f);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         m0 = fmaxf(m0, __shfl_xor_sync(0xFFFFFFFFu, m0, o));
@@ -197,125 +213,165 @@ struct QParams {
     uint8_t *row_codes;
     uint8_t *row_scales;
     float *row_tensor_scale;
+    int aligned32;  // x and every row start 32-byte aligned (256-bit loads allowed)
 };
 
 __device__ __forceinline__ float tensor_amax(const QParams &p, float *s_red) {
     return p.amax_in ? *p.amax_in : reduce_partials_max(p.partials, p.num_partials, s_red);
 }
 
-// 16-bit SR draws for the 8 consecutive output-view indices idx0 .. idx0+7
-// (idx0 % 8 == 0): one Philox block keyed on the seed at counter (idx0 >> 3).
-__device__ __forceinline__ uint4 sr_words(uint64_t idx0, uint64_t seed) {
-    return philox4x32_10(make_uint4((uint32_t)(idx0 >> 3), (uint32_t)(idx0 >> 35), 0u, 0u), (uint32_t)seed,
-                         (uint32_t)(seed >> 32));
+// The two Philox blocks that hold the 16-bit SR draws of the 16 consecutive
+// output-view indices idx0 .. idx0+15 (idx0 % 16 == 0): counters (idx0 >> 3)
+// and (idx0 >> 3) + 1, keyed on the seed.  Draw e of a block is the low (e
+// even) or high (e odd) half of word e >> 1.
+__device__ __forceinline__ void sr_words16(uint64_t idx0, const PhiloxKeys &k, uint4 &w0, uint4 &w1) {
+    const uint64_t c = idx0 >> 3;
+    w0 = philox4x32_10(make_uint4((uint32_t)c, (uint32_t)(c >> 32), 0u, 0u), k);
+    w1 = philox4x32_10(make_uint4((uint32_t)(c + 1), (uint32_t)((c + 1) >> 32), 0u, 0u), k);
 }
-__device__ __forceinline__ uint32_t rnd16_of(const uint4 &w, int e) {  // e = idx & 7
+__device__ __forceinline__ uint32_t sr_carry(const uint4 &w, int e) {  // e = idx & 7, compile-time after unrolling
     const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
-    return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+    return (e & 1) ? sr_carry_hi(word) : sr_carry_lo(word);
+}
+
+// 16 E2M1 codes of one block (element 0 in the lowest nibble of .x), from the
+// block's values and element scale; SR draws from w0 (elements 0-7) and w1
+// (8-15).  A block whose inv is 0 encodes +0 everywhere (the products are +-0,
+// and the sign bits are cleared).
+template <bool SR>
+__device__ __forceinline__ uint2 encode16(const float (&v)[16], float inv, const uint4 &w0, const uint4 &w1) {
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float r = __fmul_rn(v[i], inv);
+        q[i] = SR ? sr_e2m1_value(r, sr_carry(i < 8 ? w0 : w1, i & 7)) : r;
+    }
+    uint2 c = make_uint2(e2m1x8(q), e2m1x8(q + 8));
+    if (inv == 0.0f) {
+        c.x &= 0x77777777u;
+        c.y &= 0x77777777u;
+    }
+    return c;
+}
+
+// Loads of one 16-element block row segment: 8 (bf16) or 16 (f32) words.
+template <int LW>
+__device__ __forceinline__ void load_block(const uint8_t *src, bool a32, uint32_t (&w)[LW]) {
+    if (a32) {
+#pragma unroll
+        for (int h = 0; h < LW / 8; ++h)
+            asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(w[8 * h]), "=r"(w[8 * h + 1]), "=r"(w[8 * h + 2]), "=r"(w[8 * h + 3]), "=r"(w[8 * h + 4]),
+                           "=r"(w[8 * h + 5]), "=r"(w[8 * h + 6]), "=r"(w[8 * h + 7])
+                         : "l"(src + 32 * h));
+    } else {
+#pragma unroll
+        for (int h = 0; h < LW / 4; ++h)
+            asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(w[4 * h]), "=r"(w[4 * h + 1]), "=r"(w[4 * h + 2]), "=r"(w[4 * h + 3])
+                         : "l"(src + 16 * h));
+    }
+}
+template <typename T> __device__ __forceinline__ void unpack16(const uint32_t *w, float (&v)[16]);
+template <> __device__ __forceinline__ void unpack16<uint16_t>(const uint32_t *w, float (&v)[16]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16lo(w[i]);
+        v[2 * i + 1] = bf16hi(w[i]);
+    }
+}
+template <> __device__ __forceinline__ void unpack16<float>(const uint32_t *w, float (&v)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(w[i]);
 }
 
 // ---------------------------------------------------------------------------
-// Pass 2, rowwise: blocks of 16 along the contiguous columns.
-// Persistent CTAs walk 64-row x (32*N)-column tiles in reverse order (the amax
-// pass swept the tensor front to back, so its tail is what L2 still holds);
-// the next tile's loads are in flight while the current tile is encoded.  Warp
-// w owns rows 8w..8w+7 of a tile and each lane one 16-byte chunk of every row
-// (2 (bf16) or 4 (f32) lanes per 16-block).  Codes leave as one coalesced
-// segment per warp and row; a tile fills one half (8 of 16 bytes per atom row)
-// of each of its 128x4 scale atoms, staged in shared memory and written as
-// 8-byte pieces.  Row tiles are counted in pairs so that both halves of every
-// atom are written even when R is not a multiple of 128.
+// Pass 2, rowwise: blocks of 16 along the contiguous columns.  Each lane owns
+// one whole block of a row (one 32-byte load for bf16, two for f32), so the
+// block amax, the scale and the 16 codes (one 8-byte store) need no shuffles;
+// a warp covers 512 columns of RPW rows per tile.  Persistent CTAs walk the
+// tiles in reverse order (the amax pass swept the tensor front to back, so its
+// tail is what L2 still holds) with the next tile's loads in flight.  The four
+// scale bytes of a row within a 128x4 atom are one aligned 32-bit word held by
+// four neighbouring lanes: two shuffles gather it and one lane stores it.
+// Padding rows up to the atoms' 128-row extent and padding blocks up to their
+// 4-block width get scale 0 (their loads are zero).
 // ---------------------------------------------------------------------------
 template <typename T, bool SR>
 __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QParams p) {
-    constexpr int N = Vec<T>::N;
-    constexpr int LPB = 16 / N;          // lanes per 16-block
-    constexpr int TILE_C = 32 * N;
-    constexpr int TILE_R = 64;
-    constexpr int RPW = TILE_R / (kThreads / 32);  // rows per warp
-    constexpr int ATOMS = TILE_C / 64;   // scale atoms per tile
-    __shared__ __align__(16) uint8_t s_sc[ATOMS * 512];
+    constexpr int LW = 4 * (int)sizeof(T);          // 32-bit words per lane and row
+    constexpr int RPW = sizeof(T) == 2 ? 4 : 2;     // rows per warp per tile
+    constexpr int TILE_R = RPW * (kThreads / 32);
+    constexpr int TILE_B = 32;                      // blocks (of 16 columns) per tile row
+    __shared__ float s_inv[128];
     __shared__ float s_red[kThreads / 32];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const T *x = static_cast<const T *>(p.x);
-    const int64_t K = p.C;
-    const int64_t KB4 = (K + 63) / 64;
-    const int64_t tiles_c = (p.C + TILE_C - 1) / TILE_C;
-    const int64_t tiles_r = 2 * ((p.R + 127) / 128);
+    const uint8_t *xb = static_cast<const uint8_t *>(p.x);
+    const int64_t K = p.C, KB = K / 16, KB4 = (K + 63) / 64;
+    const int64_t tiles_c = (KB + TILE_B - 1) / TILE_B;
+    const int64_t tiles_r = ((p.R + 127) / 128) * (128 / TILE_R);
     const int64_t ntiles = tiles_c * tiles_r;
+    const bool a32 = p.aligned32 != 0;
 
-    auto load = [&](int64_t t, uint4(&buf)[RPW]) {
+    auto load = [&](int64_t t, uint32_t(&buf)[RPW][LW]) {
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t c = tc * TILE_C + lane * N;
+        const int64_t b = tc * TILE_B + lane;
         const int64_t r0 = tr * TILE_R + warp * RPW;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int64_t r = r0 + i;
-            buf[i] = (c < p.C && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+            if (b < KB && r < p.R) {
+                load_block<LW>(xb + (r * p.ld + b * 16) * (int64_t)sizeof(T), a32, buf[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < LW; ++j) buf[i][j] = 0u;
+            }
         }
     };
 
     int64_t t = ntiles - 1 - (int64_t)blockIdx.x;
-    uint4 cur[RPW], nxt[RPW];
+    uint32_t cur[RPW][LW], nxt[RPW][LW];
     if (t >= 0) load(t, cur);
     const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
     if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+    const ScaleCtx ctx = scale_ctx(s_t);
+    scale_table_init(s_inv, nullptr, s_t);
+    PhiloxKeys keys;
+    if (SR) keys = philox_keys(p.seed);
+    __syncthreads();
 
     for (; t >= 0; t -= gridDim.x) {
         const int64_t tn = t - gridDim.x;
         if (tn >= 0) load(tn, nxt);
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t c = tc * TILE_C + lane * N;
-        const bool col_ok = c < p.C;
-        const int half = (int)(tr & 1);  // which 64-row half of the 128-row atoms
+        const int64_t b = tc * TILE_B + lane, atom = b >> 2;
+        const bool col_ok = b < KB;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const int rl = warp * RPW + i;  // row within the tile
-            const int64_t r = tr * TILE_R + rl;
-            float v[N];
-            Vec<T>::unpack(cur[i], v);
+            const int64_t r = tr * TILE_R + warp * RPW + i;
+            float v[16];
+            unpack16<T>(cur[i], v);
             float m = 0.0f;
 #pragma unroll
-            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-            const BlockScale bs = block_scale(m, s_t);
-            float q[N];
-            if (SR) {
-                const uint64_t idx0 = (uint64_t)r * (uint64_t)K + (uint64_t)c;
-                const uint4 w = sr_words(idx0 & ~7ull, p.seed);
-                const int e0 = (int)(idx0 & 7);
-#pragma unroll
-                for (int j = 0; j < N; ++j)
-                    q[j] = bs.zero ? 0.0f : sr_e2m1_value(__fmul_rn(v[j], bs.inv), rnd16_of(w, e0 + j));
-            } else {
-#pragma unroll
-                for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
-            }
-            if (col_ok && r < p.R) {
-                uint8_t *dst = p.codes + r * (K / 2) + c / 2;
-                if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
-                else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
-            }
-            if ((lane % LPB) == 0) {
-                const int ra = half * TILE_R + rl, bl = lane / LPB;  // row within the 128-row atom
-                s_sc[(bl >> 2) * 512 + (ra & 31) * 16 + ((ra >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)bs.sb;
-            }
+            for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+            const uint32_t sb = block_scale_code(m, ctx);
+            const float inv = s_inv[sb];
+            uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+            if (SR) sr_words16((uint64_t)r * (uint64_t)K + (uint64_t)b * 16u, keys, w0, w1);
+            const uint2 c = encode16<SR>(v, inv, w0, w1);
+            if (col_ok && r < p.R) *reinterpret_cast<uint2 *>(p.codes + r * (K / 2) + b * 8) = c;
+            uint32_t word = sb << (8 * (lane & 3));
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+            if ((lane & 3) == 0 && atom < KB4)
+                *reinterpret_cast<uint32_t *>(p.scales + ((r >> 7) * KB4 + atom) * 512 + (r & 31) * 16 +
+                                              ((r >> 5) & 3) * 4) = word;
         }
-        __syncthreads();
-        const int64_t atom0 = tc * ATOMS;
-        for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
-            const int atom = i >> 5;
-            if (atom0 + atom < KB4) {
-                const int off = atom * 512 + (i & 31) * 16 + 8 * half;
-                uint8_t *dst = p.scales + ((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half;
-                *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(s_sc + off);
-            }
-        }
-        __syncthreads();
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) cur[i] = nxt[i];
+        for (int i = 0; i < RPW; ++i)
+#pragma unroll
+            for (int j = 0; j < LW; ++j) cur[i][j] = nxt[i][j];
     }
 }
 
@@ -324,12 +380,18 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
 // ([C x R], K = R contiguous).  CTA tile = 256 rows x (32*N) columns; warp w
 // owns rows 32w..32w+31 (two 16-row groups) and each lane N adjacent columns,
 // so every block (one column x 16 rows) sits in one thread's registers: the
-// transform, block amax and encoding need no shuffles.  A lane's 16 code bytes
-// per column (two groups) form one 16-byte unit in shared memory (each group
-// writes its 8-byte half as soon as it is encoded), placed with an xor swizzle
-// so both the scatter and the row-contiguous read-out are free of bank
-// conflicts beyond the 4-wavefront minimum.  The DUAL variant also encodes the
-// rowwise (RTN) blocks of the same rows from the same registers.
+// transform, block amax and encoding need no shuffles.  The Hadamard signs
+// are applied to the packed rows (one xor per word) before unpacking; the
+// butterfly runs unnormalised and its 1/4 is applied exactly afterwards, or,
+// with round-to-nearest and a tensor scale in the fast range, folded into the
+// element scale (inv/4, tabulated): RN(RN(z/4) * inv) = RN(z * inv/4) whenever
+// z/4 is exact, and where it is not (|z| < 2^-124) both sides give a +-0 code
+// with the sign of z.  A lane's 16 code bytes per column (two groups) form one
+// 16-byte unit in shared memory (each group writes its 8-byte half as soon as
+// it is encoded), placed with an xor swizzle so both the scatter and the
+// row-contiguous read-out are free of bank conflicts beyond the 4-wavefront
+// minimum.  The DUAL variant also encodes the rowwise (RTN) blocks of the same
+// rows from the same registers.
 // ---------------------------------------------------------------------------
 template <typename T, bool SR, bool RHT, bool DUAL>
 __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QParams p) {
@@ -343,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     __shared__ __align__(16) uint4 s_units[N * P * 32];
     __shared__ __align__(16) uint8_t s_sc[AR * AC * 512];
     __shared__ float s_red[W];
+    __shared__ float s_inv[128], s_inv4[RHT ? 128 : 1], s_inv_row[DUAL ? 128 : 1];
     constexpr int LPB = 16 / N;          // dual: lanes per rowwise 16-block
     constexpr int ARR = TR / 128;        // dual: rowwise scale-atom rows per tile
     constexpr int ACR = TC / 64;         // dual: rowwise scale-atom columns per tile
@@ -376,7 +439,20 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
         *p.tensor_scale = s_t;
         if (DUAL) *p.row_tensor_scale = s_t_row;
     }
+    const ScaleCtx ctx = scale_ctx(s_t);
+    scale_table_init(s_inv, RHT ? s_inv4 : nullptr, s_t);
+    ScaleCtx ctx_row;
+    if (DUAL) {
+        ctx_row = scale_ctx(s_t_row);
+        scale_table_init(s_inv_row, nullptr, s_t_row);
+    }
     const uint32_t signs = RHT ? rht_sign_bits(p.seed) : 0u;
+    // Quarter folded into the element scale: round-to-nearest only (a stochastic
+    // decision on a value that RN(z/4) would flush to zero can differ).
+    const bool fold = RHT && !SR && ctx.fast;
+    PhiloxKeys keys;
+    if (SR) keys = philox_keys(p.seed);
+    __syncthreads();
 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -401,21 +477,27 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
                 for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 if (LPB == 4) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-                const BlockScale bs = block_scale(m, s_t_row);
+                const uint32_t sb = block_scale_code(m, ctx_row);
+                const float inv = s_inv_row[sb];
                 float q[N];
 #pragma unroll
-                for (int j = 0; j < N; ++j) q[j] = bs.zero ? 0.0f : __fmul_rn(v[j], bs.inv);
+                for (int j = 0; j < N; ++j) q[j] = __fmul_rn(v[j], inv);
                 if (col_ok && r < p.R) {
                     uint8_t *dst = p.row_codes + r * (p.C / 2) + c / 2;
-                    if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
-                    else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
+                    if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q) & (inv == 0.0f ? 0x77777777u : ~0u);
+                    else *reinterpret_cast<uint16_t *>(dst) =
+                             (uint16_t)(e2m1x4(q[0], q[1], q[2], q[3]) & (inv == 0.0f ? 0x7777u : 0xFFFFu));
                 }
                 if ((lane % LPB) == 0) {
                     const int rl = warp * 32 + 16 * h + i, bl = lane / LPB;
                     s_scr[((rl >> 7) * ACR + (bl >> 2)) * 512 + (rl & 31) * 16 + ((rl >> 5) & 3) * 4 + (bl & 3)] =
-                        (uint8_t)bs.sb;
+                        (uint8_t)sb;
                 }
             }
+        }
+        if (RHT) {  // the sign diagonal, on the packed rows
+#pragma unroll
+            for (int i = 0; i < 16; ++i) raw[i] = xor4(raw[i], sign_mask<T>(signs, i));
         }
 #pragma unroll
         for (int j = 0; j < N; ++j) {
@@ -426,31 +508,37 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
                 Vec<T>::unpack(raw[i], t);
                 v[i] = t[j];
             }
-            if (RHT) rht16(v, signs);
-            float m = 0.0f;
+            float scale_in;  // the element scale the block's values are multiplied by
+            uint32_t sb;
+            if (RHT) {
+                fwht16(v);
+                float m = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-            const BlockScale bs = block_scale(m, s_t);
-            float q[16];
-            if (SR) {
-                const uint64_t idx0 = (uint64_t)(c + j) * (uint64_t)K + (uint64_t)rg;  // multiple of 16
-                const uint4 w0 = sr_words(idx0, p.seed), w1 = sr_words(idx0 + 8, p.seed);
+                for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+                sb = block_scale_code(__fmul_rn(m, 0.25f), ctx);  // max |z/4| = RN(max|z| / 4)
+                if (fold) {
+                    scale_in = s_inv4[sb];
+                } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    q[i] = bs.zero ? 0.0f
-                                   : sr_e2m1_value(__fmul_rn(v[i], bs.inv), rnd16_of(i < 8 ? w0 : w1, i & 7));
+                    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+                    scale_in = s_inv[sb];
+                }
             } else {
+                float m = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) q[i] = bs.zero ? 0.0f : __fmul_rn(v[i], bs.inv);
+                for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+                sb = block_scale_code(m, ctx);
+                scale_in = s_inv[sb];
             }
+            uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+            if (SR) sr_words16((uint64_t)(c + j) * (uint64_t)K + (uint64_t)rg, keys, w0, w1);  // rg % 16 == 0
+            const uint2 code = encode16<SR>(v, scale_in, w0, w1);
             {  // this group's 8 code bytes: half h of the lane's 16-byte unit for column j
                 const int qu = j * P + warp;
-                reinterpret_cast<uint2 *>(s_units)[(qu * 32 + (lane ^ (qu & 7))) * 2 + h] =
-                    make_uint2(e2m1x8(q), e2m1x8(q + 8));
+                reinterpret_cast<uint2 *>(s_units)[(qu * 32 + (lane ^ (qu & 7))) * 2 + h] = code;
             }
             const int cl = lane * N + j, gl = warp * 2 + h;
-            s_sc[((cl >> 7) * AC + (gl >> 2)) * 512 + (cl & 31) * 16 + ((cl >> 5) & 3) * 4 + (gl & 3)] =
-                (uint8_t)bs.sb;
+            s_sc[((cl >> 7) * AC + (gl >> 2)) * 512 + (cl & 31) * 16 + ((cl >> 5) & 3) * 4 + (gl & 3)] = (uint8_t)sb;
         }
     }
     __syncthreads();
@@ -682,9 +770,11 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
     }
     QParams p{a.x, a.R, a.C, a.ld, a.seed, a.amax_in, a.partials, num_partials, a.codes, a.scales,
               a.tensor_scale};
+    p.aligned32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && ((a.ld * (int64_t)sizeof(T)) % 32 == 0);
     constexpr int N = Vec<T>::N;
     if (!a.colwise) {
-        const int64_t tiles = ((a.C + 32 * N - 1) / (32 * N)) * 2 * ((a.R + 127) / 128);
+        constexpr int tile_r = sizeof(T) == 2 ? 32 : 16;  // rows per tile of quantize_rowwise_kernel
+        const int64_t tiles = ((a.C / 16 + 31) / 32) * ((a.R + 127) / 128) * (128 / tile_r);
         const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
         if (a.sr) quantize_rowwise_kernel<T, true><<<grid, kThreads, 0, s>>>(p);
         else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);

@@ -1,0 +1,122 @@
+"""The MLP block of a 12B hybrid Mamba-Transformer layer (up-projection ->
+squared ReLU -> down-projection), forward and backward, as a sequence of the
+library's C-ABI calls.
+
+Every operand of the six GEMMs is NVFP4 (aisight.pl, section "Architektura
+NVFP4 kontra ograniczenia mikroskalowania"); the Wgrad operands carry the
+16-point random Hadamard transform, and the gradient operand stochastic
+rounding (same page, section "Technologie stabilizujace proces
+treningowy").  This module only orders the calls and holds the buffers:
+argument marshalling through `binding`, all arithmetic in the CUDA library.
+
+A step, with X [M x H], W1 [F x H], W2 [H x F], dY2 [M x H] (bf16):
+  forward   X_r = rowwise(X); W1_r, W1_c = dual(W1); Y1 = X_r . W1_r^T
+            h = relu(Y1)^2 (the kernel also returns max|h| and max|RHT(h)|)
+            h_r = rowwise(h, amax supplied); W2_r, W2_c = dual(W2); Y2 = h_r . W2_r^T
+  backward  dY2_r = rowwise(dY2); dh = dY2_r . W2_c^T
+            dY2_c = colwise(dY2, RHT, SR); h_c = colwise(h, RHT, amax supplied); dW2 = dY2_c . h_c^T
+            dY1 = dh * 2 relu(Y1) (also max|dY1| and max|RHT(dY1)|)
+            dY1_r = rowwise(dY1, amax supplied); dX = dY1_r . W1_c^T
+            dY1_c = colwise(dY1, RHT, SR, amax supplied); X_c = colwise(X, RHT); dW1 = dY1_c . X_c^T
+"""
+import torch
+
+from . import binding as B
+
+SEED = 1234
+
+
+class MlpStep:
+    """Device buffers and the call sequence of one MLP block step (bf16 in and
+    out, dW in float32).  `inputs` maps X, W1, W2, dY2 to device tensors."""
+
+    def __init__(self, inputs, seed=SEED):
+        self.seed = seed
+        self.d = inputs
+        X, W1 = inputs["X"], inputs["W1"]
+        M, H = X.shape
+        F = W1.shape[0]
+        self.M, self.H, self.F = M, H, F
+        device = X.device
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.Y1 = torch.empty((M, F), **bf)
+        self.h = torch.empty_like(self.Y1)
+        self.Y2 = torch.empty((M, H), **bf)
+        self.dh = torch.empty_like(self.Y1)
+        self.dY1 = torch.empty_like(self.Y1)
+        self.dX = torch.empty((M, H), **bf)
+        self.dW1 = torch.empty((F, H), dtype=torch.float32, device=device)
+        self.dW2 = torch.empty((H, F), dtype=torch.float32, device=device)
+        self.ws = B.workspace(256, device)      # GEMM status word
+        self.qws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), device)
+        self.amax = torch.zeros(16, dtype=torch.float32, device=device)  # h, RHT(h), dY1, RHT(dY1) at 0, 4, 8, 12
+        mk = B.empty_nvfp4
+        self.q = {
+            "X_r": mk(M, H, device), "W1_r": mk(F, H, device), "W1_c": mk(H, F, device),
+            "h_r": mk(M, F, device), "W2_r": mk(H, F, device), "W2_c": mk(F, H, device),
+            "dY2_r": mk(M, H, device), "dY2_c": mk(H, M, device), "h_c": mk(F, M, device),
+            "dY1_r": mk(M, F, device), "dY1_c": mk(F, M, device), "X_c": mk(H, M, device),
+        }
+        self.launches = 0
+
+    # Each call appends (kind, algorithmic work, end event) to `ev` when given.
+    def _mark(self, ev, kind, work):
+        self.launches += B.nvfp4_last_launch_count()
+        if ev is not None:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev.append((kind, work, e))
+
+    def _quant(self, x, key, colwise=False, sr=False, rht=False, amax_in=None, ev=None, bytes_per_elem=None):
+        B.nvfp4_quantize(x, orientation=B.NVFP4_COLWISE if colwise else B.NVFP4_ROWWISE,
+                         rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, rht=rht, seed=self.seed, amax_in=amax_in,
+                         out=self.q[key], ws=self.qws)
+        self._mark(ev, "quant", x.numel() * bytes_per_elem(amax_in is not None) if bytes_per_elem else 0)
+
+    def _dual(self, x, key_r, key_c, sr=False, rht=False, ev=None, bytes_per_elem=None):
+        B.nvfp4_quantize_dual(x, col_rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, col_rht=rht, seed=self.seed,
+                              out_row=self.q[key_r], out_col=self.q[key_c], ws=self.qws)
+        self._mark(ev, "quant", x.numel() * bytes_per_elem("dual") if bytes_per_elem else 0)
+
+    def _gemm(self, a, b, out, ev=None):
+        B.nvfp4_gemm(self.q[a], self.q[b], out=out, ws=self.ws)
+        self._mark(ev, "gemm", 2 * self.q[a].rows * self.q[b].rows * self.q[a].k)
+
+    def forward(self, X=None, Y2=None, ev=None, bytes_per_elem=None):
+        d, X = self.d, (self.d["X"] if X is None else X)
+        Y2 = self.Y2 if Y2 is None else Y2
+        kw = dict(ev=ev, bytes_per_elem=bytes_per_elem)
+        self._quant(X, "X_r", **kw)
+        self._dual(d["W1"], "W1_r", "W1_c", **kw)
+        self._gemm("X_r", "W1_r", self.Y1, ev)
+        # relu^2 also returns max|h| and max|RHT(h)|: both quantisations of h skip their amax pass
+        B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=self.seed, out=self.h, amax_out=self.amax[0:1],
+                                   amax_rht_out=self.amax[4:5], ws=self.qws)
+        self._mark(ev, "relu2", self.Y1.numel())
+        self._quant(self.h, "h_r", amax_in=self.amax[0:1], **kw)
+        self._dual(d["W2"], "W2_r", "W2_c", **kw)
+        self._gemm("h_r", "W2_r", Y2, ev)
+
+    def backward(self, X=None, dY2=None, ev=None, bytes_per_elem=None):
+        d = self.d
+        X = d["X"] if X is None else X
+        dY2 = d["dY2"] if dY2 is None else dY2
+        kw = dict(ev=ev, bytes_per_elem=bytes_per_elem)
+        self._quant(dY2, "dY2_r", **kw)
+        self._gemm("dY2_r", "W2_c", self.dh, ev)
+        self._quant(dY2, "dY2_c", colwise=True, sr=True, rht=True, **kw)
+        self._quant(self.h, "h_c", colwise=True, rht=True, amax_in=self.amax[4:5], **kw)
+        self._gemm("dY2_c", "h_c", self.dW2, ev)
+        B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=self.seed, out=self.dY1, amax_out=self.amax[8:9],
+                                   amax_rht_out=self.amax[12:13], ws=self.qws)
+        self._mark(ev, "relu2", self.Y1.numel())
+        self._quant(self.dY1, "dY1_r", amax_in=self.amax[8:9], **kw)
+        self._gemm("dY1_r", "W1_c", self.dX, ev)
+        self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, amax_in=self.amax[12:13], **kw)
+        self._quant(X, "X_c", colwise=True, rht=True, **kw)
+        self._gemm("dY1_c", "X_c", self.dW1, ev)
+
+    def step(self, X=None, dY2=None, Y2=None, ev=None, bytes_per_elem=None):
+        """Forward and backward; X, dY2 and the output Y2 default to the step's own buffers."""
+        self.forward(X, Y2, ev=ev, bytes_per_elem=bytes_per_elem)
+        self.backward(X, dY2, ev=ev, bytes_per_elem=bytes_per_elem)

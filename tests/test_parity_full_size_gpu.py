@@ -1,0 +1,183 @@
+"""Full-size parity of the composite paths at the 12B layer shapes.
+
+* nvfp4_linear_fwd on the Fprop workload (X 8192x5120, W 20480x5120 bf16):
+  sampled outputs against the oracle's FP64 dot products of the oracle's own
+  quantisation of the sampled rows of X and W (GEMM on Blackwell tensor cores:
+  nerdman.de, section "Was konkret passiert ist"; format: aisight.pl, section
+  "Architektura NVFP4 kontra ograniczenia mikroskalowania").
+* The MLP block step exactly as the benchmark runs it (mlp.MlpStep, 8192 tokens,
+  hidden 5120, FFN 20480): every stage against the oracle applied to that
+  stage's own inputs -- relu^2 outputs and their producer amaxes bit-exact,
+  sampled rows of all twelve NVFP4 operands bit-exact (codes, scales, tensor
+  scale), sampled elements of all six GEMM outputs within
+  |gpu - ref| <= 1e-4 * sum|a_k b_k| (the Hadamard transform and stochastic
+  rounding of the Wgrad operands: aisight.pl, section "Technologie
+  stabilizujace proces treningowy").
+"""
+import numpy as np
+import pytest
+import torch
+
+import layout
+import oracle
+from nvfp4_bit_precision_quantize_b200 import binding as B
+from nvfp4_bit_precision_quantize_b200 import workloads as W
+from nvfp4_bit_precision_quantize_b200.mlp import MlpStep
+
+from gpu_helpers import f32_bits, first_mismatch, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def host_bits(t):
+    """bf16 device tensor -> uint16 bit patterns on the host."""
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def gpu_rows(q, rows):
+    """Codes and plain scales of selected rows of a device NVFP4 tensor."""
+    codes = q.codes[torch.from_numpy(rows).cuda()].cpu().numpy()
+    buf = q.scales.cpu().numpy()
+    scales = buf[layout.atom_offsets(q.rows, q.k)[rows]]
+    return codes, scales
+
+
+def check_operand(q, x, rows, colwise, sr, rht, seed, amax, what):
+    """Bit-exact check of sampled rows of q against the oracle's quantisation of x given amax."""
+    ts = oracle.tensor_scale(amax)
+    assert f32_bits(q.tensor_scale.cpu().numpy()[0]) == f32_bits(ts), what + ": tensor scale"
+    oc, osc = oracle.quantize_rows(x, rows, amax, colwise=colwise, sr=sr, rht=rht, seed=seed)
+    gc, gsc = gpu_rows(q, rows)
+    mm = first_mismatch(gc, oc)
+    assert mm is None, "%s: codes differ %s" % (what, mm)
+    mm = first_mismatch(gsc, osc)
+    assert mm is None, "%s: scales differ %s" % (what, mm)
+    return gc, gsc, ts
+
+
+def check_gemm_sampled(out, a_rows, a, b_rows, b, what, pairs=1200, seed=0):
+    """out[m, n] for sampled (m, n) with m in a_rows, n in b_rows, against the oracle's
+    FP64 dot products of the (already verified) operand rows a = (codes, scales, ts)."""
+    rng = np.random.default_rng(seed)
+    ia = rng.integers(0, len(a_rows), pairs)
+    ib = rng.integers(0, len(b_rows), pairs)
+    ms, ns = a_rows[ia], b_rows[ib]
+    g = out[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()].float().cpu().numpy().astype(np.float64)
+    ref, ab = oracle.gemm_sampled(a, b, ia, ib)
+    if out.dtype == torch.bfloat16:
+        # bf16 output = RN(f32 output y), |RN(y) - y| <= 2^-8 |y| and |y| <= |ref| + 1e-4 * ab
+        bound = 1e-4 * ab * (1.0 + 2.0 ** -8) + np.abs(ref) * 2.0 ** -8
+    else:
+        bound = 1e-4 * ab
+    err = np.abs(g - ref)
+    bad = err > bound
+    assert not bad.any(), "%s: %d of %d sampled outputs out of tolerance (worst %.3g of bound)" % (
+        what, int(bad.sum()), pairs, float((err / np.maximum(bound, 1e-300)).max()))
+
+
+def sample_rows(rng, n, k=40):
+    return np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, k)])).astype(np.int64)
+
+
+def test_linear_fwd_fprop_full_size(cuda_lib):
+    """nvfp4_linear_fwd at 8192 x 20480 x 5120 (the Fprop workload), f32 and bf16 outputs."""
+    w = W.fprop()
+    X, Wt = w["X"], w["W"]
+    Y = B.nvfp4_linear_fwd(to_dev(X), to_dev(Wt), y_dtype=torch.float32)
+    Y16 = B.nvfp4_linear_fwd(to_dev(X), to_dev(Wt), y_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    mr, nr = sample_rows(rng, X.shape[0]), sample_rows(rng, Wt.shape[0])
+    ax, aw = oracle.amax(X), oracle.amax(Wt)
+    xc, xs = oracle.quantize_rows(X, mr, ax)
+    wc, wsc = oracle.quantize_rows(Wt, nr, aw)
+    a = (xc, xs, oracle.tensor_scale(ax))
+    b = (wc, wsc, oracle.tensor_scale(aw))
+    check_gemm_sampled(Y, mr, a, nr, b, "Fprop f32", pairs=2000, seed=1)
+    sel = (torch.from_numpy(mr[:8]).cuda()[:, None], torch.from_numpy(nr).cuda()[None, :])
+    assert torch.equal(Y16[sel].cpu(), Y[sel].to(torch.bfloat16).cpu()), "bf16 output != RN(f32 output)"
+
+
+@pytest.fixture(scope="module")
+def mlp_run(cuda_lib):
+    """One benchmark step at full size; host copies of every stage input and output."""
+    w = W.mlp()
+    d = {k: to_dev(v) for k, v in w.items()}
+    step = MlpStep(d)
+    step.step()
+    torch.cuda.synchronize()
+    host = {k: host_bits(getattr(step, k)) for k in ("Y1", "h", "Y2", "dh", "dY1", "dX")}
+    return w, step, host
+
+
+def test_mlp_step_relu2_and_producer_amax(mlp_run):
+    w, step, host = mlp_run
+    rng = np.random.default_rng(1)
+    rows = sample_rows(rng, step.M, 64)
+    Y1, h, dh, dY1 = host["Y1"], host["h"], host["dh"], host["dY1"]
+    assert np.array_equal(h[rows], oracle.relu2_fwd(Y1[rows].ravel()).reshape(len(rows), -1))
+    assert np.array_equal(dY1[rows], oracle.relu2_bwd(dh[rows].ravel(), Y1[rows].ravel()).reshape(len(rows), -1))
+    am = step.amax.cpu().numpy()
+    assert f32_bits(am[0]) == f32_bits(oracle.amax(h))
+    assert f32_bits(am[4]) == f32_bits(oracle.amax(h, colwise=True, rht=True, seed=step.seed))
+    assert f32_bits(am[8]) == f32_bits(oracle.amax(dY1))
+    assert f32_bits(am[12]) == f32_bits(oracle.amax(dY1, colwise=True, rht=True, seed=step.seed))
+
+
+def test_mlp_step_forward(mlp_run):
+    w, step, host = mlp_run
+    rng = np.random.default_rng(2)
+    s, q = step.seed, step.q
+    # up-projection: Y1 = rowwise(X) . rowwise(W1)^T
+    xr = sample_rows(rng, step.M)
+    w1r = sample_rows(rng, step.F)
+    a = check_operand(q["X_r"], w["X"], xr, False, False, False, s, oracle.amax(w["X"]), "X_r")
+    b = check_operand(q["W1_r"], w["W1"], w1r, False, False, False, s, oracle.amax(w["W1"]), "W1_r")
+    check_gemm_sampled(step.Y1, xr, a, w1r, b, "Y1", seed=3)
+    # down-projection: Y2 = rowwise(h) . rowwise(W2)^T, h's amax from the relu^2 kernel
+    hr = sample_rows(rng, step.M)
+    w2r = sample_rows(rng, step.H)
+    a = check_operand(q["h_r"], host["h"], hr, False, False, False, s, oracle.amax(host["h"]), "h_r")
+    b = check_operand(q["W2_r"], w["W2"], w2r, False, False, False, s, oracle.amax(w["W2"]), "W2_r")
+    check_gemm_sampled(step.Y2, hr, a, w2r, b, "Y2", seed=4)
+
+
+def test_mlp_step_down_projection_backward(mlp_run):
+    w, step, host = mlp_run
+    rng = np.random.default_rng(5)
+    s, q = step.seed, step.q
+    # Dgrad: dh = rowwise(dY2) . colwise(W2)^T   ([M x H] . [F x H]^T)
+    mr = sample_rows(rng, step.M)
+    fr = sample_rows(rng, step.F)
+    a = check_operand(q["dY2_r"], w["dY2"], mr, False, False, False, s, oracle.amax(w["dY2"]), "dY2_r")
+    b = check_operand(q["W2_c"], w["W2"], fr, True, False, False, s, oracle.amax(w["W2"]), "W2_c")
+    check_gemm_sampled(step.dh, mr, a, fr, b, "dh", seed=6)
+    # Wgrad: dW2 = colwise(dY2, RHT, SR) . colwise(h, RHT)^T   ([H x M] . [F x M]^T)
+    hr = sample_rows(rng, step.H, 24)
+    fr2 = sample_rows(rng, step.F, 24)
+    a = check_operand(q["dY2_c"], w["dY2"], hr, True, True, True, s,
+                      oracle.amax(w["dY2"], colwise=True, rht=True, seed=s), "dY2_c")
+    b = check_operand(q["h_c"], host["h"], fr2, True, False, True, s,
+                      oracle.amax(host["h"], colwise=True, rht=True, seed=s), "h_c")
+    check_gemm_sampled(step.dW2, hr, a, fr2, b, "dW2", seed=7)
+
+
+def test_mlp_step_up_projection_backward(mlp_run):
+    w, step, host = mlp_run
+    rng = np.random.default_rng(8)
+    s, q = step.seed, step.q
+    dY1 = host["dY1"]
+    # Dgrad: dX = rowwise(dY1) . colwise(W1)^T   ([M x F] . [H x F]^T)
+    mr = sample_rows(rng, step.M, 24)
+    hr = sample_rows(rng, step.H, 24)
+    a = check_operand(q["dY1_r"], dY1, mr, False, False, False, s, oracle.amax(dY1), "dY1_r")
+    b = check_operand(q["W1_c"], w["W1"], hr, True, False, False, s, oracle.amax(w["W1"]), "W1_c")
+    check_gemm_sampled(step.dX, mr, a, hr, b, "dX", seed=9)
+    # Wgrad: dW1 = colwise(dY1, RHT, SR) . colwise(X, RHT)^T   ([F x M] . [H x M]^T)
+    fr = sample_rows(rng, step.F, 24)
+    hr2 = sample_rows(rng, step.H, 24)
+    a = check_operand(q["dY1_c"], dY1, fr, True, True, True, s,
+                      oracle.amax(dY1, colwise=True, rht=True, seed=s), "dY1_c")
+    b = check_operand(q["X_c"], w["X"], hr2, True, False, True, s,
+                      oracle.amax(w["X"], colwise=True, rht=True, seed=s), "X_c")
+    check_gemm_sampled(step.dW1, fr, a, hr2, b, "dW1", seed=10)

@@ -12,7 +12,8 @@ The steps: for |r| >= 1 the grid spacing is the weight of the first mantissa
 bit, so adding 2^22 - 1 - rnd16 * 2^6 to the bit pattern carries into bit 22
 exactly when the low 22 mantissa bits exceed rnd16 * 2^6; clearing them rounds.
 For |r| < 1 the same is done to 1 + |r| rounded up to binary32, then 1 is
-subtracted; results at or above 6 clamp to 6.
+subtracted.  Magnitudes are clamped to 7 first, so every result is a grid
+value or 8, and the saturating E2M1 conversion takes 8 to 6.
 """
 import numpy as np
 
@@ -25,7 +26,7 @@ def bit_pattern_sr(r, rnd16):
     """Codes from the kernels' bit-pattern SR decision (numpy restatement)."""
     r = np.asarray(r, dtype=np.float32)
     rnd16 = np.asarray(rnd16, dtype=np.uint32)
-    a = np.abs(r)
+    a = np.minimum(np.abs(r), np.float32(7.0))
     small = a < np.float32(1.0)
     base = np.where(small, np.float32(1.0), np.float32(0.0)).astype(np.float32)
     # 1 + a rounded up to binary32 (exact in float64: a * 2^23 is an integer-valued double)
@@ -34,7 +35,9 @@ def bit_pattern_sr(r, rnd16):
     carry_in = (((~rnd16) & np.uint32(0xFFFF)) << np.uint32(6)) | np.uint32(63)
     with np.errstate(over="ignore"):
         bits = (t.view(np.uint32) + carry_in) & np.uint32(0xFFC00000)
-    mag = np.minimum(bits.view(np.float32) - base, np.float32(6.0))
+    mag = bits.view(np.float32) - base
+    assert (mag <= np.float32(8.0)).all()
+    mag = np.where(mag == np.float32(8.0), np.float32(6.0), mag)  # the conversion's saturation
     codes = np.full(mag.shape, 255, dtype=np.uint8)
     for v, c in GRID_CODE.items():
         codes[mag == np.float32(v)] = c
