@@ -36,6 +36,33 @@ def shard_data_seed(base_seed, rank):
     return None if rank == 0 else base_seed + 1000 * rank
 
 
+class GradExchange:
+    """Sums each weight gradient over the ranks as soon as the step has queued the
+    GEMM that produces it, so the exchange overlaps the rest of the backward pass
+    (the down-projection's dW while the up-projection's backward runs).
+
+    ready(name, t) launches an asynchronous all-reduce of t (NCCL runs it on its
+    own stream after t's producer; gloo in the background); wait() makes the
+    caller's stream (NCCL) or the host (gloo) wait for all of them.  Every rank
+    issues the same exchanges in the same order.  On one rank both are no-ops.
+    `order` records the names in issue order."""
+
+    def __init__(self):
+        self.pending = []
+        self.order = []
+        self.active = dist.is_initialized() and dist.get_world_size() > 1
+
+    def ready(self, name, t):
+        self.order.append(name)
+        if self.active:
+            self.pending.append(dist.all_reduce(t, op=dist.ReduceOp.SUM, async_op=True))
+
+    def wait(self):
+        for w in self.pending:
+            w.wait()
+        self.pending.clear()
+
+
 def allreduce_grads(grads):
     """Sum each gradient tensor over all ranks, in place (no-op on one rank)."""
     if dist.is_initialized() and dist.get_world_size() > 1:

@@ -21,16 +21,19 @@ A step, with X [M x H], W1 [F x H], W2 [H x F], dY2 [M x H] (bf16):
 """
 import torch
 
-from . import binding as B
+from . import binding
 
 SEED = 1234
 
 
 class MlpStep:
     """Device buffers and the call sequence of one MLP block step (bf16 in and
-    out, dW in float32).  `inputs` maps X, W1, W2, dY2 to device tensors."""
+    out, dW in float32).  `inputs` maps X, W1, W2, dY2 to device tensors.
+    `lib` is the module whose calls run the step (the binding of the CUDA
+    library; tests substitute a CPU stand-in with the same call names)."""
 
-    def __init__(self, inputs, seed=SEED):
+    def __init__(self, inputs, seed=SEED, lib=binding):
+        self.B = B = lib
         self.seed = seed
         self.d = inputs
         X, W1 = inputs["X"], inputs["W1"]
@@ -61,25 +64,27 @@ class MlpStep:
 
     # Each call appends (kind, algorithmic work, end event) to `ev` when given.
     def _mark(self, ev, kind, work):
-        self.launches += B.nvfp4_last_launch_count()
+        self.launches += self.B.nvfp4_last_launch_count()
         if ev is not None:
             e = torch.cuda.Event(enable_timing=True)
             e.record()
             ev.append((kind, work, e))
 
     def _quant(self, x, key, colwise=False, sr=False, rht=False, amax_in=None, ev=None, bytes_per_elem=None):
+        B = self.B
         B.nvfp4_quantize(x, orientation=B.NVFP4_COLWISE if colwise else B.NVFP4_ROWWISE,
                          rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, rht=rht, seed=self.seed, amax_in=amax_in,
                          out=self.q[key], ws=self.qws)
         self._mark(ev, "quant", x.numel() * bytes_per_elem(amax_in is not None) if bytes_per_elem else 0)
 
     def _dual(self, x, key_r, key_c, sr=False, rht=False, ev=None, bytes_per_elem=None):
+        B = self.B
         B.nvfp4_quantize_dual(x, col_rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, col_rht=rht, seed=self.seed,
                               out_row=self.q[key_r], out_col=self.q[key_c], ws=self.qws)
         self._mark(ev, "quant", x.numel() * bytes_per_elem("dual") if bytes_per_elem else 0)
 
     def _gemm(self, a, b, out, ev=None):
-        B.nvfp4_gemm(self.q[a], self.q[b], out=out, ws=self.ws)
+        self.B.nvfp4_gemm(self.q[a], self.q[b], out=out, ws=self.ws)
         self._mark(ev, "gemm", 2 * self.q[a].rows * self.q[b].rows * self.q[a].k)
 
     def forward(self, X=None, Y2=None, ev=None, bytes_per_elem=None):
@@ -90,14 +95,16 @@ class MlpStep:
         self._dual(d["W1"], "W1_r", "W1_c", **kw)
         self._gemm("X_r", "W1_r", self.Y1, ev)
         # relu^2 also returns max|h| and max|RHT(h)|: both quantisations of h skip their amax pass
-        B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=self.seed, out=self.h, amax_out=self.amax[0:1],
-                                   amax_rht_out=self.amax[4:5], ws=self.qws)
+        self.B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=self.seed, out=self.h, amax_out=self.amax[0:1],
+                                        amax_rht_out=self.amax[4:5], ws=self.qws)
         self._mark(ev, "relu2", self.Y1.numel())
         self._quant(self.h, "h_r", amax_in=self.amax[0:1], **kw)
         self._dual(d["W2"], "W2_r", "W2_c", **kw)
         self._gemm("h_r", "W2_r", Y2, ev)
 
-    def backward(self, X=None, dY2=None, ev=None, bytes_per_elem=None):
+    def backward(self, X=None, dY2=None, ev=None, bytes_per_elem=None, grad_ready=None):
+        """grad_ready(name, tensor), if given, is called as soon as the GEMM producing
+        a weight gradient is queued: dW2 first, then dW1."""
         d = self.d
         X = d["X"] if X is None else X
         dY2 = d["dY2"] if dY2 is None else dY2
@@ -107,16 +114,20 @@ class MlpStep:
         self._quant(dY2, "dY2_c", colwise=True, sr=True, rht=True, **kw)
         self._quant(self.h, "h_c", colwise=True, rht=True, amax_in=self.amax[4:5], **kw)
         self._gemm("dY2_c", "h_c", self.dW2, ev)
-        B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=self.seed, out=self.dY1, amax_out=self.amax[8:9],
-                                   amax_rht_out=self.amax[12:13], ws=self.qws)
+        if grad_ready:
+            grad_ready("dW2", self.dW2)
+        self.B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=self.seed, out=self.dY1, amax_out=self.amax[8:9],
+                                        amax_rht_out=self.amax[12:13], ws=self.qws)
         self._mark(ev, "relu2", self.Y1.numel())
         self._quant(self.dY1, "dY1_r", amax_in=self.amax[8:9], **kw)
         self._gemm("dY1_r", "W1_c", self.dX, ev)
         self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, amax_in=self.amax[12:13], **kw)
         self._quant(X, "X_c", colwise=True, rht=True, **kw)
         self._gemm("dY1_c", "X_c", self.dW1, ev)
+        if grad_ready:
+            grad_ready("dW1", self.dW1)
 
-    def step(self, X=None, dY2=None, Y2=None, ev=None, bytes_per_elem=None):
+    def step(self, X=None, dY2=None, Y2=None, ev=None, bytes_per_elem=None, grad_ready=None):
         """Forward and backward; X, dY2 and the output Y2 default to the step's own buffers."""
         self.forward(X, Y2, ev=ev, bytes_per_elem=bytes_per_elem)
-        self.backward(X, dY2, ev=ev, bytes_per_elem=bytes_per_elem)
+        self.backward(X, dY2, ev=ev, bytes_per_elem=bytes_per_elem, grad_ready=grad_ready)
