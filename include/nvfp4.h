@@ -187,6 +187,21 @@ NVFP4_API nvfp4_status nvfp4_quantize_dual(const void *x, nvfp4_dtype dtype, int
 NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
                         int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * nvfp4_gemm_mx -- the same GEMM on MXFP4 operands, the comparison format of
+ * aisight.pl, section "Architektura NVFP4 kontra ograniczenia
+ * mikroskalowania" (32-element blocks, power-of-two E8M0 scales, no tensor
+ * scale): C[M x N] = A . B^T with A = [M x K], B = [N x K] as written by
+ * nvfp4_quantize_mx (codes as for NVFP4, scales nvfp4_mx_scales_bytes(rows, K)
+ * bytes in that layout); tensor_scale is ignored.  Products of E2M1 values
+ * and E8M0 block scales accumulate in FP32 on the tensor cores
+ * (kind::mxf4.block_scale.block32) and the epilogue writes c_dtype (f32, or
+ * bf16 by round-to-nearest-even) with leading dimension ldc elements.
+ * Requirements, workspace and errors as nvfp4_gemm.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
+                                     int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Workspace bytes at these sizes: nvfp4_linear_workspace_size serves both
  * nvfp4_linear_fwd and nvfp4_linear_bwd (the larger of the two footprints);
  * nvfp4_linear_fwd_workspace_size is what nvfp4_linear_fwd alone needs (the

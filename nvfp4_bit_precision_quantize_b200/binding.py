@@ -36,7 +36,8 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_status_string", "nvfp4_linear_fwd_noalloc", "nvfp4_selftest_wait_timeout",
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
-           "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size")
+           "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
+           "nvfp4_gemm_mx")
 
 
 class CTensor(C.Structure):
@@ -69,6 +70,7 @@ def load():
         "nvfp4_quantize_workspace_size": (sz, []),
         "nvfp4_quantize": (i32, [vp, i32, i64, i64, i64, i32, i32, i32, u64, vp, tp, vp, sz, vp]),
         "nvfp4_gemm": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
+        "nvfp4_gemm_mx": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
         "nvfp4_linear_workspace_size": (sz, [i64, i64, i64]),
         "nvfp4_linear_fwd_workspace_size": (sz, [i64, i64, i64]),
         "nvfp4_linear_fwd": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]),
@@ -175,9 +177,9 @@ def _workspace(ws):
     return _nbytes(ws) if ws is not None else 0
 
 
-def _quantised(name, q, scales_bytes):
+def _quantised(name, q, scales_bytes, tensor_scale=True):
     """The buffers of an NVFP4 / MXFP4 tensor are device memory and large enough."""
-    _on_device(q.codes, q.scales, q.tensor_scale)
+    _on_device(q.codes, q.scales, *([q.tensor_scale] if tensor_scale else []))
     for part, t in (("codes", q.codes), ("scales", q.scales)):
         if not t.is_contiguous():
             raise ValueError("%s.%s must be contiguous" % (name, part))
@@ -185,7 +187,8 @@ def _quantised(name, q, scales_bytes):
         raise ValueError("%s.codes: %d bytes, need %d" % (name, _nbytes(q.codes), q.rows * (q.k // 2)))
     if _nbytes(q.scales) < scales_bytes:
         raise ValueError("%s.scales: %d bytes, need %d" % (name, _nbytes(q.scales), scales_bytes))
-    _scalar_out(name + ".tensor_scale", q.tensor_scale)
+    if tensor_scale:
+        _scalar_out(name + ".tensor_scale", q.tensor_scale)
 
 
 @dataclass
@@ -270,7 +273,7 @@ def nvfp4_quantize_mx(x, orientation=NVFP4_ROWWISE, out=None, stream=None):
                                                 device=x.device),
                              tensor_scale=None, rows=rows, k=k)
     _on_device(x)
-    _quantised("out", out, nvfp4_mx_scales_bytes(out.rows, out.k))
+    _quantised("out", out, nvfp4_mx_scales_bytes(out.rows, out.k), tensor_scale=False)
     ct = out.c()
     _ok(load().nvfp4_quantize_mx(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), orientation, C.byref(ct),
                                  _stream(stream)), "nvfp4_quantize_mx")
@@ -317,6 +320,24 @@ def nvfp4_gemm(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
     st = load().nvfp4_gemm(C.byref(ca), C.byref(cb), _ptr(out), _dtype_code(out.dtype), out.stride(0), _ptr(ws),
                            _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_gemm")
+    return out
+
+
+def nvfp4_gemm_mx(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None):
+    """C = A . B^T for MXFP4 tensors A [M x K], B [N x K] (from nvfp4_quantize_mx)."""
+    M, N = A.rows, B.rows
+    out = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=A.codes.device)
+    ws = ws if ws is not None else workspace(256, A.codes.device)
+    _quantised("A", A, nvfp4_mx_scales_bytes(A.rows, A.k), tensor_scale=False)
+    _quantised("B", B, nvfp4_mx_scales_bytes(B.rows, B.k), tensor_scale=False)
+    _rows("out", out)
+    if out.shape[0] < M or out.shape[1] < N:
+        raise ValueError("out: shape %s, need at least (%d, %d)" % (tuple(out.shape), M, N))
+    _on_device(out, ws)
+    ca, cb = A.c(), B.c()
+    st = load().nvfp4_gemm_mx(C.byref(ca), C.byref(cb), _ptr(out), _dtype_code(out.dtype), out.stride(0), _ptr(ws),
+                              _workspace(ws), _stream(stream))
+    _ok(st, "nvfp4_gemm_mx")
     return out
 
 

@@ -193,7 +193,7 @@ nvfp4_status quantize_impl(const void *x, nvfp4_dtype dtype, int64_t R, int64_t 
 }
 
 nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype, int64_t ldc,
-                       void *ws, cudaStream_t stream, int *launches) {
+                       void *ws, cudaStream_t stream, int *launches, bool mx = false) {
     GemmArgs g;
     g.a_codes = A->codes;
     g.a_scales = A->scales;
@@ -208,6 +208,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nv
     g.c_bf16 = c_dtype == NVFP4_DTYPE_BF16;
     g.ldc = ldc;
     g.status = static_cast<int *>(ws);
+    g.mx = mx;
     return from_cuda(launch_gemm(g, stream, launches));
 }
 
@@ -364,6 +365,22 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, n
     if (A->rows == 0 || B->rows == 0) return call.done(NVFP4_OK);  // nothing to launch
     if ((st = check_device()) != NVFP4_OK) return st;
     return call.done(gemm_impl(A, B, C, c_dtype, ldc, workspace, stream, &call.launches));
+}
+
+nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype, int64_t ldc,
+                           void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    Call call(__func__);
+    if (!A || !B) return NVFP4_ERR_INVALID_ARG;
+    // the same checks as nvfp4_gemm, without the tensor scales (MXFP4 has none)
+    nvfp4_tensor a = *A, b = *B;
+    static float placeholder;
+    a.tensor_scale = b.tensor_scale = &placeholder;
+    nvfp4_status st = validate_gemm(&a, &b, C, c_dtype, ldc, workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    if (A->rows == 0 || B->rows == 0) return call.done(NVFP4_OK);
+    if ((st = check_device()) != NVFP4_OK) return st;
+    a.tensor_scale = b.tensor_scale = nullptr;
+    return call.done(gemm_impl(&a, &b, C, c_dtype, ldc, workspace, stream, &call.launches, true));
 }
 
 nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,

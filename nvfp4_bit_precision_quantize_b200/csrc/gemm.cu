@@ -73,6 +73,14 @@ constexpr int GROUP_N = 8;                     // tile columns per raster group
 // 10-12, K-major, N >> 3 at bits 17-22, UE4M3 scales (bit 23 = 0), M >> 4 at
 // bits 24-28 (M = 256 across the pair), scale-factor byte ids 0, dense K = 64.
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// MXFP4 (kind::mxf4, blocks of 32): the same fields with UE8M0 scales (bit 23).
+// Each K = 64 step reads two scale bytes per row out of a 4-byte TMEM word; the
+// byte they start at (0 or 2) goes in bits 29-30 (A) and 4-5 (B).
+constexpr uint32_t IDESC_MX = IDESC | (1u << 23);
+__host__ __device__ constexpr uint32_t idesc_mx(uint32_t sf_byte) { return IDESC_MX | (sf_byte << 29) | (sf_byte << 4); }
+// Scale atoms (128 rows x 4 bytes) per 256-k stage and 128-row tile: one per 64 k
+// for NVFP4 (16-element blocks), one per 128 k for MXFP4 (32-element blocks).
+template <bool MX> constexpr int kAtomsPerStage = MX ? 2 : 4;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -186,15 +194,25 @@ __device__ __forceinline__ void tc_cp_scales_if(uint32_t issue, uint32_t taddr, 
         "r"(taddr), "l"(sdesc)
         : "memory");
 }
+template <bool MX>
 __device__ __forceinline__ void tc_mma_if(uint32_t issue, uint32_t d, uint64_t a, uint64_t b, uint32_t sfa,
-                                          uint32_t sfb, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "setp.ne.b32 q, %7, 0;\n\t"
-        "@q tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(IDESC), "r"(acc), "r"(sfa), "r"(sfb), "r"(issue)
-        : "memory");
+                                          uint32_t sfb, uint32_t acc, uint32_t idesc) {
+    if (MX)
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "setp.ne.b32 q, %7, 0;\n\t"
+            "@q tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(issue)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "setp.ne.b32 q, %7, 0;\n\t"
+            "@q tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+            "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb), "r"(issue)
+            : "memory");
 }
 // Arrives on the barrier at the same offset in both CTAs once every MMA issued so far has completed.
 __device__ __forceinline__ void tc_commit_pair_if(uint32_t issue, uint32_t bar) {
@@ -274,7 +292,7 @@ struct KParams {
     void *C;
     int64_t ldc;
     int M, N, K;
-    int kb4;    // scale atoms per 128-row tile (= K / 64)
+    int kbs;    // scale atoms per 128-row tile (K / 64 for NVFP4, ceil(K / 128) for MXFP4)
     int kfull;  // full 256-k stages (= K / 256)
     int ktail;  // 64-k steps in a last, partial stage (= (K % 256) / 64)
     int c_bf16;
@@ -292,6 +310,7 @@ __device__ __forceinline__ void tile_coords(const KParams &p, int t, int &mt, in
     nt = g * GROUP_N + (r - mt * gw);
 }
 
+template <bool MX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
@@ -349,7 +368,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 int mt, nt;
                 tile_coords(p, t, mt, nt);
                 const int m0 = mt * BM + 128 * (int)rank, n0 = nt * BN;
-                const int ya = (m0 / 128) * p.kb4, yb = (n0 / 128) * p.kb4;
+                constexpr int APS = kAtomsPerStage<MX>;
+                constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 3 * APS * 512;  // bytes per CTA per stage
+                const int ya = (m0 / 128) * p.kbs, yb = (n0 / 128) * p.kbs;
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag)) {
                         ok = false;
@@ -359,13 +380,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t full_leader = mapa(bar_full + 8 * s, 0);
                     // Out-of-range rows, columns and atoms are zero-filled and still
                     // counted, so every stage brings exactly STAGE_BYTES per CTA.
-                    if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_BYTES);
+                    if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_TX);
                     tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
                     tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, ya + kt * 4, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * 4, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, ya + kt * APS, policy);
+                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * APS, policy);
                     tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES + 2048, &map_sfb, full_leader, 0,
-                                  yb + p.kb4 + kt * 4, policy);
+                                  yb + p.kbs + kt * APS, policy);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
@@ -399,7 +420,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
                     // +128 for B's second 128-row tile, +2 per 64-k step of codes.
                     const int steps = kt < kfull ? 4 : ktail;
-                    if (steps == 4) {
+                    if (MX) {
+                        // one atom per two 64-k steps; step j reads bytes 2 (j % 2), 2 (j % 2) + 1
+                        for (int j = 0; j < (steps + 1) / 2; ++j) {
+                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                        }
+                        for (int j = 0; j < steps; ++j)
+                            tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1),
+                                          (acc | (uint32_t)j) ? 1u : 0u, idesc_mx(2u * (uint32_t)(j & 1)));
+                    } else if (steps == 4) {
                         if (lane == 0) {
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
@@ -407,10 +438,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                                 tc_cp_scales_if(1u, sf + 16 + 8 * j, dsb + 32 * j);
                                 tc_cp_scales_if(1u, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                             }
-                            tc_mma_if(1u, tmem, da, db, sf, sf + 16, acc);
+                            tc_mma_if<MX>(1u, tmem, da, db, sf, sf + 16, acc, IDESC);
 #pragma unroll
                             for (int j = 1; j < 4; ++j)
-                                tc_mma_if(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u);
+                                tc_mma_if<MX>(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u, IDESC);
                         }
                         __syncwarp();
                     } else {
@@ -420,8 +451,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
                         for (int j = 0; j < steps; ++j)
-                            tc_mma_if(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
-                                      (acc | (uint32_t)j) ? 1u : 0u);
+                            tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
+                                          (acc | (uint32_t)j) ? 1u : 0u, IDESC);
                     }
                     acc = 1;
                     tc_commit_pair_if(issue, bar_empty + 8 * s);
@@ -480,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t tbase = tmem + ((q * 32u) << 16) + 128u * (uint32_t)h;
         uint64_t policy;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
-        const float scale = __fmul_rn(*p.tsa, *p.tsb);
+        const float scale = MX ? 1.0f : __fmul_rn(*p.tsa, *p.tsb);  // MXFP4 has no tensor scale
         int tile_i = 0;
         for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
             bool ok = mbar_wait(bar_accf, tile_i & 1, abort_flag);
@@ -618,32 +649,27 @@ bool make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_
 }
 
 // A scale buffer as rows of one 512-byte atom (128 words): [atoms x 128] words,
-// box = 4 atoms (one 256-k stage of one 128-row tile).
-bool make_scale_map(CUtensorMap *map, const uint8_t *scales, int64_t rows, int64_t K) {
+// box = the atoms of one 256-k stage of one 128-row tile (4 NVFP4, 2 MXFP4).
+bool make_scale_map(CUtensorMap *map, const uint8_t *scales, int64_t rows, int64_t kbs, int box_atoms) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const int64_t atoms = ((rows + 127) / 128) * (K / 64);
+    const int64_t atoms = ((rows + 127) / 128) * kbs;
     cuuint64_t dims[2] = {128u, (cuuint64_t)atoms};
     cuuint64_t strides[1] = {512u};
-    cuuint32_t box[2] = {128u, 4u};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_atoms};
     cuuint32_t estr[2] = {1u, 1u};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
-    const size_t esz = a.c_bf16 ? 2 : 4;
-    if (a.M == 0 || a.N == 0) return cudaSuccess;
-    if (a.K == 0) {
-        ++*launches;
-        return cudaMemset2DAsync(a.C, (size_t)a.ldc * esz, 0, (size_t)a.N * esz, (size_t)a.M, s);
-    }
+template <bool MX>
+cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
+    const int kbs = MX ? (int)((a.K + 127) / 128) : (int)(a.K / 64);
     CUtensorMap map_a, map_b, map_sfa, map_sfb;
     if (!make_codes_map(&map_a, a.a_codes, a.M, a.K) || !make_codes_map(&map_b, a.b_codes, a.N, a.K) ||
-        !make_scale_map(&map_sfa, a.a_scales, a.M, a.K) || !make_scale_map(&map_sfb, a.b_scales, a.N, a.K))
+        !make_scale_map(&map_sfa, a.a_scales, a.M, kbs, kAtomsPerStage<MX>) ||
+        !make_scale_map(&map_sfb, a.b_scales, a.N, kbs, kAtomsPerStage<MX>))
         return cudaErrorInvalidValue;
     constexpr int kMaxDev = 64;
     static int max_clusters[kMaxDev] = {};
@@ -652,7 +678,7 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
     if (!max_clusters[dev]) {
-        e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        e = cudaFuncSetAttribute(gemm_nvfp4_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         // Pairs that can be resident at once (one CTA per SM).
         cudaLaunchConfig_t cfg = {};
@@ -660,7 +686,7 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
         cfg.blockDim = dim3(THREADS);
         cfg.dynamicSmemBytes = SMEM_BYTES;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel<MX>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = num_sms() / 2;
         }
@@ -674,7 +700,7 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.M = (int)a.M;
     p.N = (int)a.N;
     p.K = (int)a.K;
-    p.kb4 = (int)(a.K / 64);
+    p.kbs = kbs;
     p.kfull = (int)(a.K / BK);
     p.ktail = (int)((a.K % BK) / 64);
     p.c_bf16 = a.c_bf16 ? 1 : 0;
@@ -683,9 +709,21 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.status = a.status;
     const int pairs = std::min(p.num_tiles, max_clusters[dev]);
-    gemm_nvfp4_kernel<<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, p);
+    gemm_nvfp4_kernel<MX><<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, p);
     ++*launches;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
+    const size_t esz = a.c_bf16 ? 2 : 4;
+    if (a.M == 0 || a.N == 0) return cudaSuccess;
+    if (a.K == 0) {
+        ++*launches;
+        return cudaMemset2DAsync(a.C, (size_t)a.ldc * esz, 0, (size_t)a.N * esz, (size_t)a.M, s);
+    }
+    return a.mx ? launch_gemm_t<true>(a, s, launches) : launch_gemm_t<false>(a, s, launches);
 }
 
 }  // namespace nvfp4

@@ -54,6 +54,7 @@ struct GemmArgs {
     bool c_bf16;
     int64_t ldc;
     int *status;
+    bool mx = false;  // MXFP4 operands (E8M0 scales per 32 k, no tensor scales)
 };
 
 // Each launcher adds the number of kernels it launched to *launches.

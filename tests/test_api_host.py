@@ -112,6 +112,22 @@ def test_gemm_rejections(lib):
     assert g(A=_tensor(0, 256)) == E.NVFP4_OK                         # empty: nothing to do
 
 
+def test_gemm_mx_rejections(lib):
+    E = binding
+    A, Bt = _tensor(256, 256), _tensor(256, 256)
+    Bt.tensor_scale = None                                             # MXFP4 tensors carry no tensor scale
+    p = C.c_void_p
+    g = lambda A=A, Bt=Bt, Cp=0x40000, dt=0, ldc=256, ws=0x50000: lib.nvfp4_gemm_mx(  # noqa: E731
+        C.byref(A), C.byref(Bt), p(Cp), dt, ldc, p(ws) if ws else None, 256, None)
+    assert g(A=_tensor(256, 96)) == E.NVFP4_ERR_SHAPE                 # K mismatch
+    assert g(A=_tensor(256, 96), Bt=_tensor(256, 96)) == E.NVFP4_ERR_SHAPE  # K % 64
+    assert g(Cp=0) == E.NVFP4_ERR_INVALID_ARG
+    assert g(Cp=0x40004) == E.NVFP4_ERR_ALIGNMENT
+    assert g(ws=0) == E.NVFP4_ERR_WORKSPACE
+    assert g(dt=3) == E.NVFP4_ERR_INVALID_ARG
+    assert g(A=_tensor(0, 256)) == E.NVFP4_OK
+
+
 def test_linear_rejections(lib):
     E = binding
     ws = lib.nvfp4_linear_workspace_size(128, 128, 128)
