@@ -202,6 +202,35 @@ NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, 
 NVFP4_API nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C, nvfp4_dtype c_dtype,
                                      int64_t ldc, void *workspace, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * nvfp4_gemm_relu2_fwd / nvfp4_gemm_relu2_bwd -- the MLP block's GEMMs next to
+ * its squared ReLU, with the activation applied in the GEMM's epilogue.  The
+ * 12B model's MLP (hyper.ai, "NVIDIA revolutioniert
+ * KI-Praetrainingsgeschwindigkeit mit 4-Bit-Genauigkeit") runs up-projection ->
+ * relu^2 -> down-projection in NVFP4 (aisight.pl, section "Architektura NVFP4
+ * kontra ograniczenia mikroskalowania").  Both take NVFP4 A [M x K] and B [N x K]
+ * as nvfp4_gemm and compute y = bf16(A . B^T * sA * sB) (round to nearest
+ * even), then:
+ *   fwd: Y = y and H = relu(y) * relu(y)      (the up-projection and h)
+ *   bwd: dY = y * (2 * relu(Y)), Y the forward's y, y not stored
+ *        (the down-projection's Dgrad dh, and dY1 of the up-projection)
+ * each product in binary32 then bf16 round-to-nearest-even, bit-identical to
+ * nvfp4_gemm followed by nvfp4_relu2_fwd / nvfp4_relu2_bwd.  They also write
+ * *amax_out = max |H| (|dY|) and *amax_rht_out = max |RHT(H)| (|RHT(dY)|),
+ * the 16-point random Hadamard transform of `seed` down 16-row groups (as
+ * nvfp4_relu2_fwd_amax_rht), for the two quantisations of that output.
+ * Y, H, dY: contiguous bf16 [M x N], 16-byte aligned, device memory.
+ * Requires M and N multiples of 256, K % 64 == 0, K > 0.  workspace: >=
+ * nvfp4_quantize_dual_workspace_size() bytes, 16-byte aligned, zeroed status
+ * word.  Two launches.  Errors as nvfp4_gemm; NVFP4_ERR_SHAPE for other M, N.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_relu2_fwd(const nvfp4_tensor *A, const nvfp4_tensor *B, void *Y, void *H,
+                                            uint64_t seed, float *amax_out, float *amax_rht_out, void *workspace,
+                                            size_t ws_bytes, cudaStream_t stream);
+NVFP4_API nvfp4_status nvfp4_gemm_relu2_bwd(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *Y, void *dY,
+                                            uint64_t seed, float *amax_out, float *amax_rht_out, void *workspace,
+                                            size_t ws_bytes, cudaStream_t stream);
+
 /* Workspace bytes at these sizes: nvfp4_linear_workspace_size serves both
  * nvfp4_linear_fwd and nvfp4_linear_bwd (the larger of the two footprints);
  * nvfp4_linear_fwd_workspace_size is what nvfp4_linear_fwd alone needs (the

@@ -37,7 +37,7 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
            "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
-           "nvfp4_gemm_mx")
+           "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd")
 
 
 class CTensor(C.Structure):
@@ -71,6 +71,8 @@ def load():
         "nvfp4_quantize": (i32, [vp, i32, i64, i64, i64, i32, i32, i32, u64, vp, tp, vp, sz, vp]),
         "nvfp4_gemm": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
         "nvfp4_gemm_mx": (i32, [tp, tp, vp, i32, i64, vp, sz, vp]),
+        "nvfp4_gemm_relu2_fwd": (i32, [tp, tp, vp, vp, u64, vp, vp, vp, sz, vp]),
+        "nvfp4_gemm_relu2_bwd": (i32, [tp, tp, vp, vp, u64, vp, vp, vp, sz, vp]),
         "nvfp4_linear_workspace_size": (sz, [i64, i64, i64]),
         "nvfp4_linear_fwd_workspace_size": (sz, [i64, i64, i64]),
         "nvfp4_linear_fwd": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp, sz, vp]),
@@ -339,6 +341,39 @@ def nvfp4_gemm_mx(A, B, out_dtype=torch.bfloat16, out=None, ws=None, stream=None
                               _workspace(ws), _stream(stream))
     _ok(st, "nvfp4_gemm_mx")
     return out
+
+
+def _gemm_relu2(name, A, B, y, out, seed, amax_out, amax_rht_out, ws, stream):
+    M, N = A.rows, B.rows
+    dev = A.codes.device
+    out = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    amax_out = _amax_buffer(amax_out, dev)
+    amax_rht_out = _amax_buffer(amax_rht_out, dev)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), dev)
+    _quantised("A", A, nvfp4_scales_bytes(A.rows, A.k))
+    _quantised("B", B, nvfp4_scales_bytes(B.rows, B.k))
+    for nm, t in (("y", y), ("out", out)):
+        _dense(nm, t, shape=(M, N), dtype=torch.bfloat16)
+    _on_device(y, out, amax_out, amax_rht_out, ws)
+    ca, cb = A.c(), B.c()
+    st = getattr(load(), name)(C.byref(ca), C.byref(cb), _ptr(y), _ptr(out), seed, _ptr(amax_out),
+                               _ptr(amax_rht_out), _ptr(ws), _workspace(ws), _stream(stream))
+    _ok(st, name)
+    return out, amax_out, amax_rht_out
+
+
+def nvfp4_gemm_relu2_fwd(A, B, seed=1234, y=None, h=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
+    """y = bf16(A . B^T sA sB) and h = relu(y)^2 (bf16), with max|h| and max|RHT(h)|.
+    Returns (y, h, amax, amax_rht)."""
+    y = y if y is not None else torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    h, a0, a1 = _gemm_relu2("nvfp4_gemm_relu2_fwd", A, B, y, h, seed, amax_out, amax_rht_out, ws, stream)
+    return y, h, a0, a1
+
+
+def nvfp4_gemm_relu2_bwd(A, B, y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None, stream=None):
+    """dY = bf16(bf16(A . B^T sA sB) * 2 relu(y)) for the forward's y, with max|dY| and
+    max|RHT(dY)|.  Returns (dY, amax, amax_rht)."""
+    return _gemm_relu2("nvfp4_gemm_relu2_bwd", A, B, y, out, seed, amax_out, amax_rht_out, ws, stream)
 
 
 def _linear_operands(X, W):

@@ -383,6 +383,57 @@ nvfp4_status nvfp4_gemm_mx(const nvfp4_tensor *A, const nvfp4_tensor *B, void *C
     return call.done(gemm_impl(&a, &b, C, c_dtype, ldc, workspace, stream, &call.launches, true));
 }
 
+namespace {
+nvfp4_status gemm_relu2_impl(const char *name, int epi, const nvfp4_tensor *A, const nvfp4_tensor *B, void *C,
+                             void *aux, uint64_t seed, float *amax_out, float *amax_rht_out, void *workspace,
+                             size_t ws_bytes, cudaStream_t stream) {
+    Call call(name);
+    nvfp4_status st = validate_gemm(A, B, C, NVFP4_DTYPE_BF16, B ? B->rows : 0, workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    const int64_t M = A->rows, N = B->rows;
+    if (M == 0 || N == 0 || A->k == 0 || M % 256 != 0 || N % 256 != 0) return NVFP4_ERR_SHAPE;
+    if (!aux || !amax_out || !amax_rht_out) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(aux) || !aligned16(amax_out) || !aligned16(amax_rht_out)) return NVFP4_ERR_ALIGNMENT;
+    if (ws_bytes < kDualWorkspace) return NVFP4_ERR_WORKSPACE;
+    if ((st = check_device()) != NVFP4_OK) return st;
+    GemmArgs g;
+    g.a_codes = A->codes;
+    g.a_scales = A->scales;
+    g.a_ts = A->tensor_scale;
+    g.b_codes = B->codes;
+    g.b_scales = B->scales;
+    g.b_ts = B->tensor_scale;
+    g.M = M;
+    g.N = N;
+    g.K = A->k;
+    g.C = C;
+    g.c_bf16 = true;
+    g.ldc = N;
+    g.status = static_cast<int *>(workspace);
+    g.epi = epi;
+    g.aux = aux;
+    g.seed = seed;
+    g.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    g.amax_out = amax_out;
+    g.amax_rht_out = amax_rht_out;
+    return call.done(from_cuda(launch_gemm(g, stream, &call.launches)));
+}
+}  // namespace
+
+nvfp4_status nvfp4_gemm_relu2_fwd(const nvfp4_tensor *A, const nvfp4_tensor *B, void *Y, void *H, uint64_t seed,
+                                  float *amax_out, float *amax_rht_out, void *workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    return gemm_relu2_impl(__func__, GEMM_EPI_RELU2_FWD, A, B, Y, H, seed, amax_out, amax_rht_out, workspace,
+                           ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_gemm_relu2_bwd(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *Y, void *dY,
+                                  uint64_t seed, float *amax_out, float *amax_rht_out, void *workspace,
+                                  size_t ws_bytes, cudaStream_t stream) {
+    return gemm_relu2_impl(__func__, GEMM_EPI_RELU2_BWD, A, B, dY, const_cast<void *>(Y), seed, amax_out,
+                           amax_rht_out, workspace, ws_bytes, stream);
+}
+
 nvfp4_status nvfp4_linear_fwd(const void *X, const void *W, void *Y, int64_t M, int64_t N, int64_t K,
                               nvfp4_dtype dtype, nvfp4_dtype y_dtype, void *workspace, size_t ws_bytes,
                               cudaStream_t stream) {

@@ -65,6 +65,28 @@ __device__ __forceinline__ uint32_t rht_sign_bits(uint64_t seed) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {  // round to nearest even
+    uint32_t w;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
+    return w;
+}
+
+// Squared ReLU of the MLP block and its derivative on bf16 pairs: one binary32
+// operation each, then bf16 round-to-nearest-even; relu(y) = +0 for y <= 0.
+//   h = relu(y) * relu(y)        dy = dh * (2 * relu(y))
+__device__ __forceinline__ float relu(float y) { return y > 0.0f ? y : 0.0f; }
+__device__ __forceinline__ uint32_t relu2_pair(uint32_t y) {
+    const float a = relu(bf16lo(y)), b = relu(bf16hi(y));
+    return pack_bf16x2(__fmul_rn(a, a), __fmul_rn(b, b));
+}
+__device__ __forceinline__ uint32_t drelu2_pair(uint32_t dh, uint32_t y) {
+    const float ga = __fmul_rn(2.0f, relu(bf16lo(y))), gb = __fmul_rn(2.0f, relu(bf16hi(y)));
+    return pack_bf16x2(__fmul_rn(bf16lo(dh), ga), __fmul_rn(bf16hi(dh), gb));
+}
+__device__ __forceinline__ float absmax_pair(float m, uint32_t w) {
+    return fmaxf(m, fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w))));
+}
+
 template <typename T> struct Vec;  // 16-byte vector of T, unpacked to floats
 template <> struct Vec<uint16_t> {  // bf16 bit patterns
     static constexpr int N = 8;

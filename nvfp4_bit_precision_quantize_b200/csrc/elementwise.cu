@@ -13,26 +13,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ float relu(float y) { return y > 0.0f ? y : 0.0f; }
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    uint32_t w;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
-    return w;
-}
 __device__ __forceinline__ uint16_t bf16_of(float f) { return (uint16_t)(pack_bf16x2(f, 0.0f) & 0xFFFFu); }
-
-__device__ __forceinline__ uint32_t relu2_pair(uint32_t y) {
-    const float a = relu(bf16lo(y)), b = relu(bf16hi(y));
-    return pack_bf16x2(__fmul_rn(a, a), __fmul_rn(b, b));
-}
-__device__ __forceinline__ uint32_t drelu2_pair(uint32_t dh, uint32_t y) {
-    const float ga = __fmul_rn(2.0f, relu(bf16lo(y))), gb = __fmul_rn(2.0f, relu(bf16hi(y)));
-    return pack_bf16x2(__fmul_rn(bf16lo(dh), ga), __fmul_rn(bf16hi(dh), gb));
-}
-
-__device__ __forceinline__ float absmax_pair(float m, uint32_t w) {
-    return fmaxf(m, fmaxf(fabsf(bf16lo(w)), fabsf(bf16hi(w))));
-}
 // Block-wide max written as this CTA's partial.
 __device__ __forceinline__ void write_partial(float m, float *partials) {
     __shared__ float s_red[kThreads / 32];
@@ -223,6 +204,13 @@ cudaError_t launch_relu2_amax_rht(const void *dh, const void *y, void *out, int6
                                                                partials + kMaxPartials);
     amax_reduce2_kernel<<<1, kThreads, 0, s>>>(partials, partials + kMaxPartials, (int)grid, amax_out, amax_rht_out);
     *launches += 2;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_out, float *amax_rht_out, cudaStream_t s,
+                                int *launches) {
+    amax_reduce2_kernel<<<1, kThreads, 0, s>>>(partials, partials + kMaxPartials, count, amax_out, amax_rht_out);
+    ++*launches;
     return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ constexpr int WAITER_WARP = 10;
 // Hardware named barriers (64 threads: the waiter warp and the MMA warp).
 constexpr uint32_t NB_ACC = 1;     // accumulator free for the next tile
 constexpr uint32_t NB_STAGE0 = 2;  // NB_STAGE0 + s: stage s loaded
+constexpr uint32_t NB_EPI = NB_STAGE0 + STAGES;  // the 8 epilogue warps (fused amax reduction)
 constexpr uint32_t TMEM_COLS = 512;            // accumulator 256 columns + scales 48 columns, rounded up
 constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
@@ -298,6 +299,10 @@ struct KParams {
     int c_bf16;
     int tiles_m, tiles_n, num_tiles;
     int *status;
+    int epi;          // GEMM_EPI_* (internal.h)
+    void *aux;        // relu^2 forward: h (out); backward: the forward's y (in)
+    uint64_t seed;    // Hadamard signs of the fused amax
+    float *partials;  // per CTA: max |out| at [cta], max |RHT(out)| at [kMaxPartials + cta]
 };
 
 // Tile t -> (tile row, tile column).  Tile columns form bands of GROUP_N; inside
@@ -356,6 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t smem_base = smem_u32(smem);
     const int num_kt = p.kfull + (p.ktail ? 1 : 0);
+    float epi_m0 = 0.0f, epi_m1 = 0.0f;  // epilogue, fused relu^2: max |out|, max |H16 D out| (unscaled)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -512,6 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint64_t policy;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
         const float scale = MX ? 1.0f : __fmul_rn(*p.tsa, *p.tsb);  // MXFP4 has no tensor scale
+        const uint32_t row_sign = p.epi != GEMM_EPI_PLAIN ? ((rht_sign_bits(p.seed) >> (lane & 15)) & 1u) << 31 : 0u;
         int tile_i = 0;
         for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
             bool ok = mbar_wait(bar_accf, tile_i & 1, abort_flag);
@@ -544,6 +551,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
                     if (!row_ok) continue;
                     uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + c0;
+                    if (p.epi != GEMM_EPI_PLAIN) {
+                        // Squared ReLU (or its derivative) of the bf16 result, stored, with
+                        // the running max |out| and max |H16 D out| down the 16-row groups
+                        // (lanes 0-15 and 16-31 hold consecutive rows): the butterfly runs
+                        // across lanes, lower lane a + b, upper lane a - b, strides 1..8.
+                        uint16_t *aux = static_cast<uint16_t *>(p.aux) + (int64_t)row * p.ldc + c0;
+                        const bool fwd = p.epi == GEMM_EPI_RELU2_FWD;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            uint32_t o[4];
+                            if (fwd) {
+                                st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) o[k] = relu2_pair(w[4 * j + k]);
+                                st_global_v4(aux + 8 * j, o[0], o[1], o[2], o[3], policy);
+                            } else {
+                                const uint4 y = *reinterpret_cast<const uint4 *>(aux + 8 * j);
+                                o[0] = drelu2_pair(w[4 * j], y.x);
+                                o[1] = drelu2_pair(w[4 * j + 1], y.y);
+                                o[2] = drelu2_pair(w[4 * j + 2], y.z);
+                                o[3] = drelu2_pair(w[4 * j + 3], y.w);
+                                st_global_v4(dst + 8 * j, o[0], o[1], o[2], o[3], policy);
+                            }
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                float v = (k & 1) ? bf16hi(o[k >> 1]) : bf16lo(o[k >> 1]);
+                                epi_m0 = fmaxf(epi_m0, fabsf(v));
+                                v = __uint_as_float(__float_as_uint(v) ^ row_sign);
+#pragma unroll
+                                for (int hs = 1; hs < 16; hs <<= 1) {
+                                    const float pv = __shfl_xor_sync(0xFFFFFFFFu, v, hs);
+                                    v = (lane & hs) ? __fsub_rn(pv, v) : __fadd_rn(v, pv);
+                                }
+                                epi_m1 = fmaxf(epi_m1, fabsf(v));
+                            }
+                        }
+                        continue;
+                    }
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
@@ -609,6 +654,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                 }
             }
+        }
+    }
+
+    if (p.epi != GEMM_EPI_PLAIN && warp >= 2 && warp < 2 + EPI_WARPS) {
+        // this CTA's partials of the fused amax: warps, then the 8 epilogue warps
+        float *red = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 128);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            epi_m0 = fmaxf(epi_m0, __shfl_xor_sync(0xFFFFFFFFu, epi_m0, o));
+            epi_m1 = fmaxf(epi_m1, __shfl_xor_sync(0xFFFFFFFFu, epi_m1, o));
+        }
+        if (lane == 0) {
+            red[warp - 2] = epi_m0;
+            red[EPI_WARPS + warp - 2] = epi_m1;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(NB_EPI), "r"(32 * EPI_WARPS) : "memory");
+        if (warp == 2 && lane == 0) {
+            float a = 0.0f, b = 0.0f;
+            for (int i = 0; i < EPI_WARPS; ++i) {
+                a = fmaxf(a, red[i]);
+                b = fmaxf(b, red[EPI_WARPS + i]);
+            }
+            p.partials[blockIdx.x] = a;
+            p.partials[kMaxPartials + blockIdx.x] = __fmul_rn(b, 0.25f);  // max |z / 4| = RN(max |z| / 4)
         }
     }
 
@@ -708,9 +777,18 @@ cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.tiles_n = (int)((a.N + BN - 1) / BN);
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.status = a.status;
+    p.epi = a.epi;
+    p.aux = a.aux;
+    p.seed = a.seed;
+    p.partials = a.partials;
     const int pairs = std::min(p.num_tiles, max_clusters[dev]);
     gemm_nvfp4_kernel<MX><<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, p);
     ++*launches;
+    if (a.epi != GEMM_EPI_PLAIN) {
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_amax_reduce2(a.partials, 2 * pairs, a.amax_out, a.amax_rht_out, s, launches);
+    }
     return cudaGetLastError();
 }
 

@@ -55,7 +55,20 @@ struct GemmArgs {
     int64_t ldc;
     int *status;
     bool mx = false;  // MXFP4 operands (E8M0 scales per 32 k, no tensor scales)
+    // Fused squared-ReLU epilogue (bf16 output, M and N multiples of 256, M < 2^31):
+    //   GEMM_EPI_RELU2_FWD: C = y = bf16(acc), aux (out) = relu(y)^2
+    //   GEMM_EPI_RELU2_BWD: C = bf16(bf16(acc) * 2 relu(aux)), aux (in) = the forward's y
+    // with max |relu output| and max |RHT(relu output)| (16-point transform of
+    // `seed` down 16-row groups) written to amax_out[0] and amax_out[1] through
+    // partials (2 * kMaxPartials floats).
+    int epi = 0;
+    void *aux = nullptr;
+    uint64_t seed = 0;
+    float *partials = nullptr;
+    float *amax_out = nullptr;
+    float *amax_rht_out = nullptr;
 };
+constexpr int GEMM_EPI_PLAIN = 0, GEMM_EPI_RELU2_FWD = 1, GEMM_EPI_RELU2_BWD = 2;
 
 // Each launcher adds the number of kernels it launched to *launches.
 cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches);
@@ -68,6 +81,10 @@ cudaError_t launch_relu2_fwd(const void *y, void *h, int64_t n, float *amax_out,
                              int *launches);
 cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n, float *amax_out, float *partials,
                              cudaStream_t s, int *launches);
+
+// max over per-CTA partials (plain at partials, RHT at partials + kMaxPartials) -> *amax_out, *amax_rht_out
+cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_out, float *amax_rht_out, cudaStream_t s,
+                                int *launches);
 
 // One bounded wait on an mbarrier nothing arrives on; records the timeout status.
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);

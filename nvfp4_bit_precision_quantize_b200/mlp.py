@@ -10,14 +10,19 @@ treningowy").  This module only orders the calls and holds the buffers:
 argument marshalling through `binding`, all arithmetic in the CUDA library.
 
 A step, with X [M x H], W1 [F x H], W2 [H x F], dY2 [M x H] (bf16):
-  forward   X_r = rowwise(X); W1_r, W1_c = dual(W1); Y1 = X_r . W1_r^T
-            h = relu(Y1)^2 (the kernel also returns max|h| and max|RHT(h)|)
+  forward   X_r = rowwise(X); W1_r, W1_c = dual(W1)
+            Y1 = X_r . W1_r^T and h = relu(Y1)^2 from one GEMM (the epilogue also
+            returns max|h| and max|RHT(h)|)
             h_r = rowwise(h, amax supplied); W2_r, W2_c = dual(W2); Y2 = h_r . W2_r^T
-  backward  dY2_r = rowwise(dY2); dh = dY2_r . W2_c^T
+  backward  dY2_r = rowwise(dY2)
+            dY1 = (dY2_r . W2_c^T) * 2 relu(Y1) from one GEMM (the epilogue applies the
+            derivative to the bf16 dh, which is never stored, and returns max|dY1| and
+            max|RHT(dY1)|)
             dY2_c = colwise(dY2, RHT, SR); h_c = colwise(h, RHT, amax supplied); dW2 = dY2_c . h_c^T
-            dY1 = dh * 2 relu(Y1) (also max|dY1| and max|RHT(dY1)|)
             dY1_r = rowwise(dY1, amax supplied); dX = dY1_r . W1_c^T
             dY1_c = colwise(dY1, RHT, SR, amax supplied); X_c = colwise(X, RHT); dW1 = dY1_c . X_c^T
+With fused=False the two squared-ReLU steps run as their own kernels after
+plain GEMMs (dh stored), with the same results bit for bit.
 """
 import torch
 
@@ -32,9 +37,10 @@ class MlpStep:
     `lib` is the module whose calls run the step (the binding of the CUDA
     library; tests substitute a CPU stand-in with the same call names)."""
 
-    def __init__(self, inputs, seed=SEED, lib=binding):
+    def __init__(self, inputs, seed=SEED, lib=binding, fused=True):
         self.B = B = lib
         self.seed = seed
+        self.fused = fused
         self.d = inputs
         X, W1 = inputs["X"], inputs["W1"]
         M, H = X.shape
@@ -45,7 +51,7 @@ class MlpStep:
         self.Y1 = torch.empty((M, F), **bf)
         self.h = torch.empty_like(self.Y1)
         self.Y2 = torch.empty((M, H), **bf)
-        self.dh = torch.empty_like(self.Y1)
+        self.dh = None if fused else torch.empty_like(self.Y1)  # the fused Dgrad epilogue never stores dh
         self.dY1 = torch.empty_like(self.Y1)
         self.dX = torch.empty((M, H), **bf)
         self.dW1 = torch.empty((F, H), dtype=torch.float32, device=device)
@@ -93,11 +99,16 @@ class MlpStep:
         kw = dict(ev=ev, bytes_per_elem=bytes_per_elem)
         self._quant(X, "X_r", **kw)
         self._dual(d["W1"], "W1_r", "W1_c", **kw)
-        self._gemm("X_r", "W1_r", self.Y1, ev)
         # relu^2 also returns max|h| and max|RHT(h)|: both quantisations of h skip their amax pass
-        self.B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=self.seed, out=self.h, amax_out=self.amax[0:1],
-                                        amax_rht_out=self.amax[4:5], ws=self.qws)
-        self._mark(ev, "relu2", self.Y1.numel())
+        if self.fused:
+            self.B.nvfp4_gemm_relu2_fwd(self.q["X_r"], self.q["W1_r"], seed=self.seed, y=self.Y1, h=self.h,
+                                        amax_out=self.amax[0:1], amax_rht_out=self.amax[4:5], ws=self.qws)
+            self._mark(ev, "gemm", 2 * self.M * self.F * self.H)
+        else:
+            self._gemm("X_r", "W1_r", self.Y1, ev)
+            self.B.nvfp4_relu2_fwd_amax_rht(self.Y1, seed=self.seed, out=self.h, amax_out=self.amax[0:1],
+                                            amax_rht_out=self.amax[4:5], ws=self.qws)
+            self._mark(ev, "relu2", self.Y1.numel())
         self._quant(self.h, "h_r", amax_in=self.amax[0:1], **kw)
         self._dual(d["W2"], "W2_r", "W2_c", **kw)
         self._gemm("h_r", "W2_r", Y2, ev)
@@ -110,15 +121,22 @@ class MlpStep:
         dY2 = d["dY2"] if dY2 is None else dY2
         kw = dict(ev=ev, bytes_per_elem=bytes_per_elem)
         self._quant(dY2, "dY2_r", **kw)
-        self._gemm("dY2_r", "W2_c", self.dh, ev)
+        # dY1 = dh * 2 relu(Y1), with max|dY1| and max|RHT(dY1)| for its two quantisations
+        if self.fused:
+            self.B.nvfp4_gemm_relu2_bwd(self.q["dY2_r"], self.q["W2_c"], self.Y1, seed=self.seed, out=self.dY1,
+                                        amax_out=self.amax[8:9], amax_rht_out=self.amax[12:13], ws=self.qws)
+            self._mark(ev, "gemm", 2 * self.M * self.F * self.H)
+        else:
+            self._gemm("dY2_r", "W2_c", self.dh, ev)
         self._quant(dY2, "dY2_c", colwise=True, sr=True, rht=True, **kw)
         self._quant(self.h, "h_c", colwise=True, rht=True, amax_in=self.amax[4:5], **kw)
         self._gemm("dY2_c", "h_c", self.dW2, ev)
         if grad_ready:
             grad_ready("dW2", self.dW2)
-        self.B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=self.seed, out=self.dY1, amax_out=self.amax[8:9],
-                                        amax_rht_out=self.amax[12:13], ws=self.qws)
-        self._mark(ev, "relu2", self.Y1.numel())
+        if not self.fused:
+            self.B.nvfp4_relu2_bwd_amax_rht(self.dh, self.Y1, seed=self.seed, out=self.dY1, amax_out=self.amax[8:9],
+                                            amax_rht_out=self.amax[12:13], ws=self.qws)
+            self._mark(ev, "relu2", self.Y1.numel())
         self._quant(self.dY1, "dY1_r", amax_in=self.amax[8:9], **kw)
         self._gemm("dY1_r", "W1_c", self.dX, ev)
         self._quant(self.dY1, "dY1_c", colwise=True, sr=True, rht=True, amax_in=self.amax[12:13], **kw)

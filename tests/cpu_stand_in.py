@@ -99,3 +99,21 @@ def nvfp4_relu2_fwd_amax_rht(y, seed=1234, out=None, amax_out=None, amax_rht_out
 def nvfp4_relu2_bwd_amax_rht(dh, y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None):
     calls.append("relu2_bwd")
     _relu2_amax(oracle.relu2_bwd(_bits(dh).ravel(), _bits(y).ravel()), seed, out, amax_out, amax_rht_out)
+
+
+def nvfp4_gemm_relu2_fwd(A, B, seed=1234, y=None, h=None, amax_out=None, amax_rht_out=None, ws=None):
+    calls.append("gemm_relu2_fwd")
+    ref, _ = oracle.gemm((A.codes.numpy(), A.scales.numpy(), A.tensor_scale.item()),
+                         (B.codes.numpy(), B.scales.numpy(), B.tensor_scale.item()))
+    y.copy_(torch.from_numpy(ref).to(torch.bfloat16))
+    _relu2_amax(oracle.relu2_fwd(_bits(y).ravel()), seed, h, amax_out, amax_rht_out)
+    return y, h, amax_out, amax_rht_out
+
+
+def nvfp4_gemm_relu2_bwd(A, B, y, seed=1234, out=None, amax_out=None, amax_rht_out=None, ws=None):
+    calls.append("gemm_relu2_bwd")
+    ref, _ = oracle.gemm((A.codes.numpy(), A.scales.numpy(), A.tensor_scale.item()),
+                         (B.codes.numpy(), B.scales.numpy(), B.tensor_scale.item()))
+    dh = _bits(torch.from_numpy(ref).to(torch.bfloat16))
+    _relu2_amax(oracle.relu2_bwd(dh.ravel(), _bits(y).ravel()), seed, out, amax_out, amax_rht_out)
+    return out, amax_out, amax_rht_out

@@ -104,9 +104,11 @@ def test_two_rank_mlp_step_exchange():
         local.append((st.dW1, st.dW2))
     for rank, calls, order, dW1, dW2 in res:
         assert order == ["dW2", "dW1"]
-        assert calls.count("gemm") == 6
+        gemms = [i for i, c in enumerate(calls) if c.startswith("gemm")]
+        assert len(gemms) == 6
         i2 = calls.index("exchange dW2")
-        assert calls[i2 - 1] == "gemm" and calls.index("relu2_bwd") > i2      # overlaps the up-projection bwd
+        assert calls[i2 - 1] == "gemm"
+        assert sum(1 for i in gemms if i > i2) == 2                          # overlaps the up-projection bwd
         assert calls[-1] == "exchange dW1" and calls[-2] == "gemm"
         assert torch.equal(dW1, local[0][0] + local[1][0])
         assert torch.equal(dW2, local[0][1] + local[1][1])
