@@ -461,6 +461,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     mx_us = m0.elapsed_time(m1) / 20 * 1e3
 
+    # MXFP4 GEMM (the pages' comparison format) at the Fprop shape on random MXFP4
+    # operands, timed apart from the step
+    mx_gemm = mxfp4_gemm_timing(B, device)
+
     pk, src = peaks()
     if rank == 0:
         g = stats["gemm"]
@@ -508,6 +512,7 @@ def run_ours(args):
                                "peak": pk["hbm_gbs"],
                                "frac": hten.numel() * MX_BYTES / (mx_us * 1e-6) / 1e9 / pk["hbm_gbs"],
                                "bytes_per_elem": MX_BYTES},
+            "mxfp4_gemm": dict(mx_gemm, peak=fp4_peak, frac=mx_gemm["achieved"] / fp4_peak),
             "breakdown_ms_per_step": {k: v[0] / args.steps for k, v in stats.items()},
             "e2e": {"value": nproc * GEMM_FLOPS / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -519,6 +524,35 @@ def run_ours(args):
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line))
     dp.finish()
+
+
+def mxfp4_gemm_timing(B, device, M=M_TOK, N=FFN, K=HID, n=20):
+    """nvfp4_gemm_mx at M x N x K (bf16 out) on random MXFP4 operands: CUDA events over n launches."""
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+
+    def operand(rows):
+        return B.NVFP4Tensor(
+            codes=torch.randint(0, 256, (rows, K // 2), dtype=torch.uint8, device=device, generator=g),
+            scales=torch.randint(118, 136, (B.nvfp4_mx_scales_bytes(rows, K),), dtype=torch.uint8, device=device,
+                                 generator=g),
+            tensor_scale=None, rows=rows, k=K)
+    a, b = operand(M), operand(N)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    ws = B.workspace(256, device)
+    for _ in range(3):
+        B.nvfp4_gemm_mx(a, b, out=out, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        B.nvfp4_gemm_mx(a, b, out=out, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    B.nvfp4_check(ws)
+    ms = e0.elapsed_time(e1) / n
+    return {"shape": "%dx%dx%d bf16 out" % (M, N, K), "launch_ms": ms, "achieved": 2 * M * N * K / ms / 1e9,
+            "unit": "TFLOP/s"}
 
 
 def run_profile_case(case):

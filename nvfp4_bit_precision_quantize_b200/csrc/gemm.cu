@@ -1,11 +1,12 @@
-// gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a tensor cores.
+// gemm.cu -- block-scaled NVFP4 (and MXFP4) GEMM on the sm_100a tensor cores.
 //
 // C[M x N] = (A . B^T) * sA * sB with A [M x K], B [N x K] both K-major NVFP4:
 // packed E2M1 codes, one E4M3 scale per 16 k (the 128x4 scale atoms written by
 // the quantiser), one FP32 tensor scale each.  4-bit GEMMs on Blackwell
 // tensor cores: nerdman.de, "Nvidia drueckt KI-Training auf 4 Bit runter",
 // section "Was konkret passiert ist"; format: aisight.pl, section
-// "Architektura NVFP4 kontra ograniczenia mikroskalowania".
+// "Architektura NVFP4 kontra ograniczenia mikroskalowania" (which also gives
+// MXFP4, 32-element blocks with power-of-two scales, as the comparison).
 //
 // Persistent kernel on CTA pairs (cluster of 2 SMs).  A pair owns a 256 x 256
 // output tile at a time: CTA rank r holds A rows [128r, 128r+128) of the tile
@@ -24,12 +25,19 @@
 //   warp 10            waiter (leader): polls the stage-full and
 //                      accumulator-free barriers and relays each event to the
 //                      MMA warp through a hardware named barrier, so that the
-//                      issuing warp never waits on shared memory (its latency
-//                      is high while the tensor cores stream operands);
+//                      issuing warp never waits on shared memory;
 //   warps 2..9         epilogue: two warps per 32-lane TMEM quarter, each
-//                      reading 128 accumulator columns into registers
-//                      (tcgen05.ld), then handing TMEM back to the leader
-//                      before it scales by sA*sB and stores f32 / bf16.
+//                      reading 128 accumulator columns (tcgen05.ld), handing
+//                      TMEM back to the leader, then scaling by sA*sB and
+//                      writing f32 / bf16 through a swizzled 4 KB
+//                      shared-memory chunk and a TMA store (32 rows x 128
+//                      bytes per chunk; per-row stores from registers cost
+//                      several microseconds per tile here).
+// Scale copies through four extra warps (tcgen05.st from shared memory into
+// per-stage TMEM slots, keeping the MMA warp's pipe free of copies) were
+// measured slower: the extra hop on every stage's refill path cost more than
+// the ~24 tensor-pipe cycles per copy it saves, with five stages in flight.
+// TMEM: accumulator columns [0, 256), then the 48 scale columns of one stage.
 // Tiles are visited in groups of 8 tile columns so that the pairs running at
 // the same time share A and B panels in L2.  Every mbarrier wait is bounded
 // (about 2 s of %globaltimer); on expiry the CTA records
@@ -52,18 +60,23 @@ constexpr int A_BYTES = 128 * BK / 2;          // 16 KB: this CTA's 128 A rows
 constexpr int B_BYTES = 128 * BK / 2;          // 16 KB: this CTA's 128 B rows
 constexpr int SFA_BYTES = (BK / 64) * 512;     // 2 KB: scale atoms of this CTA's A rows
 constexpr int SFB_BYTES = 2 * (BK / 64) * 512; // 4 KB: scale atoms of all 256 B rows
+constexpr int SF_OFF = A_BYTES + B_BYTES;      // scale atoms inside a stage: A, B rows 0-127, B rows 128-255
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128B swizzle");
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr int THREADS = 352;                    // producer, MMA, 8 epilogue warps, waiter
 constexpr int EPI_WARPS = 8;
-constexpr int WAITER_WARP = 10;
+constexpr int CHUNK_BYTES = 4096;               // epilogue staging per warp: 32 rows x 128 bytes
+constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
+constexpr int BAR_OFF = STAGING_OFF + EPI_WARPS * CHUNK_BYTES;
+constexpr int BAR_BYTES = 512;
+constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+constexpr int THREADS = 352;                    // producer, MMA, 8 epilogue warps, waiter
+constexpr int MMA_WARP = 1, EPI_WARP0 = 2, WAITER_WARP = 10;
 // Hardware named barriers (64 threads: the waiter warp and the MMA warp).
 constexpr uint32_t NB_ACC = 1;     // accumulator free for the next tile
 constexpr uint32_t NB_STAGE0 = 2;  // NB_STAGE0 + s: stage s loaded
 constexpr uint32_t NB_EPI = NB_STAGE0 + STAGES;  // the 8 epilogue warps (fused amax reduction)
-constexpr uint32_t TMEM_COLS = 512;            // accumulator 256 columns + scales 48 columns, rounded up
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 20000000ull;
@@ -269,13 +282,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void st_global_v4(void *dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                             uint64_t policy) {
-    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(a), "r"(b), "r"(c),
-                 "r"(d), "l"(policy)
-                 : "memory");
-}
-
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart (SBO); LBO unused; version 1 (sm_100).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
@@ -288,10 +294,41 @@ __device__ __forceinline__ uint64_t sdesc_scales(uint32_t saddr) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
+// TMA load into this CTA's shared memory, completing on this CTA's own barrier.
+__device__ __forceinline__ void tma_load_own(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y,
+                                             uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+// TMA store of a shared-memory box (bulk async-group completion).
+__device__ __forceinline__ void tma_store(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the TMA engine.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Byte offset of 16-byte unit u of row r in a 32-row x 128-byte chunk laid out
+// with the TMA 128-byte swizzle (unit index xor row % 8): a warp's 16-byte
+// accesses of one unit index cover all banks.
+__device__ __forceinline__ uint32_t chunk_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
 struct KParams {
     const float *tsa, *tsb;
-    void *C;
-    int64_t ldc;
     int M, N, K;
     int kbs;    // scale atoms per 128-row tile (K / 64 for NVFP4, ceil(K / 128) for MXFP4)
     int kfull;  // full 256-k stages (= K / 256)
@@ -300,7 +337,6 @@ struct KParams {
     int tiles_m, tiles_n, num_tiles;
     int *status;
     int epi;          // GEMM_EPI_* (internal.h)
-    void *aux;        // relu^2 forward: h (out); backward: the forward's y (in)
     uint64_t seed;    // Hadamard signs of the fused amax
     float *partials;  // per CTA: max |out| at [cta], max |RHT(out)| at [kMaxPartials + cta]
 };
@@ -315,26 +351,65 @@ __device__ __forceinline__ void tile_coords(const KParams &p, int t, int &mt, in
     nt = g * GROUP_N + (r - mt * gw);
 }
 
+// One epilogue chunk (32 rows x 128 bytes, row = lane) from registers into the
+// warp's staging buffer and out through a TMA store.  The previous store of
+// this warp must have finished reading the buffer first.
+__device__ __forceinline__ void store_chunk(const CUtensorMap *map, uint32_t stg, const uint32_t (&w)[32], int lane,
+                                            int x, int y, bool write) {
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 8; ++u) st_shared_v4(stg + chunk_off(lane, u), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0 && write) {
+        tma_store(map, stg, x, y);
+        bulk_commit();
+    }
+}
+
+// Running max |v| and max |H16 D v| of one bf16 pair per lane, the transform
+// down the 16-row groups held by lanes 0-15 and 16-31 (lower lane a + b, upper
+// lane a - b, strides 1, 2, 4, 8): the fused relu^2 epilogue's two amaxes.
+__device__ __forceinline__ void amax_pair_rht(uint32_t o, uint32_t row_sign, int lane, float &m0, float &m1) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        float v = k ? bf16hi(o) : bf16lo(o);
+        m0 = fmaxf(m0, fabsf(v));
+        v = __uint_as_float(__float_as_uint(v) ^ row_sign);
+#pragma unroll
+        for (int hs = 1; hs < 16; hs <<= 1) {
+            const float pv = __shfl_xor_sync(0xFFFFFFFFu, v, hs);
+            v = (lane & hs) ? __fsub_rn(pv, v) : __fadd_rn(v, pv);
+        }
+        m1 = fmaxf(m1, fabsf(v));
+    }
+}
+
 template <bool MX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                      const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_aux,
                       const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    const uint32_t bar_full = smem_u32(bars);                // [S] leader: both CTAs' bytes of a stage
-    const uint32_t bar_empty = smem_u32(bars + STAGES);      // [S] each CTA: MMAs reading the stage done
-    const uint32_t bar_accf = smem_u32(bars + 2 * STAGES);   // each CTA: accumulator complete
-    const uint32_t bar_acce = smem_u32(bars + 2 * STAGES + 1);  // leader: accumulator read (8 epilogue warps)
-    const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2); // leader: every MMA done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
+    const uint32_t bar_full = smem_u32(bars);                    // [S] leader: both CTAs' bytes of a stage
+    const uint32_t bar_empty = smem_u32(bars + STAGES);          // [S] each CTA: MMAs reading the stage done
+    const uint32_t bar_accf = smem_u32(bars + 2 * STAGES);       // each CTA: accumulator complete
+    const uint32_t bar_acce = smem_u32(bars + 2 * STAGES + 1);   // leader: accumulator read (16 epilogue warps)
+    const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2);  // leader: every MMA done
+    const uint32_t bar_epi = smem_u32(bars + 2 * STAGES + 3);    // [8] each CTA: an epilogue warp's aux chunk
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3 + EPI_WARPS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *stop_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // waiter -> MMA warp, per tile
+    float *red = reinterpret_cast<float *>(tmem_slot + 4);                      // fused amax: 2 x 8 warps
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cta_rank();
     const int cid = (int)cluster_id_x(), ncl = (int)nclusters_x();
+    constexpr int APS = kAtomsPerStage<MX>;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -344,11 +419,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         mbar_init(bar_accf, 1);
         mbar_init(bar_acce, 2 * EPI_WARPS);
         mbar_init(bar_drain, 1);
+        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(bar_epi + 8 * w, 1);
         *abort_flag = 0;
         *stop_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         __syncwarp();
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(TMEM_COLS)
@@ -370,12 +446,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
             uint32_t s = 0, ph = 0;
             bool ok = true;
+            constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 3 * APS * 512;  // bytes per CTA per stage
             for (int t = cid; t < p.num_tiles && ok; t += ncl) {
                 int mt, nt;
                 tile_coords(p, t, mt, nt);
                 const int m0 = mt * BM + 128 * (int)rank, n0 = nt * BN;
-                constexpr int APS = kAtomsPerStage<MX>;
-                constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 3 * APS * 512;  // bytes per CTA per stage
                 const int ya = (m0 / 128) * p.kbs, yb = (n0 / 128) * p.kbs;
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, abort_flag)) {
@@ -385,14 +460,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t st = smem_base + s * STAGE_BYTES;
                     const uint32_t full_leader = mapa(bar_full + 8 * s, 0);
                     // Out-of-range rows, columns and atoms are zero-filled and still
-                    // counted, so every stage brings exactly STAGE_BYTES per CTA.
+                    // counted, so every stage brings exactly STAGE_TX bytes per CTA.
                     if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_TX);
                     tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
                     tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES, &map_sfa, full_leader, 0, ya + kt * APS, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * APS, policy);
-                    tma_load_pair(st + A_BYTES + B_BYTES + SFA_BYTES + 2048, &map_sfb, full_leader, 0,
-                                  yb + p.kbs + kt * APS, policy);
+                    tma_load_pair(st + SF_OFF, &map_sfa, full_leader, 0, ya + kt * APS, policy);
+                    tma_load_pair(st + SF_OFF + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * APS, policy);
+                    tma_load_pair(st + SF_OFF + SFA_BYTES + 2048, &map_sfb, full_leader, 0, yb + p.kbs + kt * APS,
+                                  policy);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
@@ -401,16 +476,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             // This CTA's loads complete on the leader's barriers; the leader drains them.
         }
-    } else if (warp == 1) {
+    } else if (warp == MMA_WARP) {
         if (rank == 0) {
             // ---------------- MMA issuer (leader's warp 1, lane 0 issues) ----------------
             const uint32_t issue = lane == 0 ? 1u : 0u;
             const int kfull = p.kfull, ktail = p.ktail;
             uint32_t s = 0, ph = 0;
-            int consumed = 0, tile_i = 0;
+            int consumed = 0;
             // Every event this warp waits for comes from the waiter warp through a
             // named barrier: the loop below reads no shared memory per stage.
-            for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
+            for (int t = cid; t < p.num_tiles; t += ncl) {
                 named_sync(NB_ACC);
                 if (*stop_flag) break;  // written by the waiter before the barrier
                 tc_fence_after();
@@ -420,45 +495,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     named_sync(NB_STAGE0 + s);
                     const uint32_t sa = smem_base + s * STAGE_BYTES;
                     const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + A_BYTES);
-                    const uint64_t dsa = sdesc_scales(sa + A_BYTES + B_BYTES);
-                    const uint64_t dsb = sdesc_scales(sa + A_BYTES + B_BYTES + SFA_BYTES);
+                    const uint64_t dsa = sdesc_scales(sa + SF_OFF);
+                    const uint64_t dsb = sdesc_scales(sa + SF_OFF + SFA_BYTES);
                     const uint32_t sf = tmem + TMEM_SF;
                     // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
                     // +128 for B's second 128-row tile, +2 per 64-k step of codes.
+                    // Scales: A atom j at sf + 4 j, B atoms at sf + 16 + 8 j (rows 0-127)
+                    // and sf + 20 + 8 j (rows 128-255); MXFP4 atom j serves steps 2j, 2j+1.
                     const int steps = kt < kfull ? 4 : ktail;
-                    if (MX) {
-                        // one atom per two 64-k steps; step j reads bytes 2 (j % 2), 2 (j % 2) + 1
-                        for (int j = 0; j < (steps + 1) / 2; ++j) {
-                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
-                        }
-                        for (int j = 0; j < steps; ++j)
-                            tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1),
-                                          (acc | (uint32_t)j) ? 1u : 0u, idesc_mx(2u * (uint32_t)(j & 1)));
-                    } else if (steps == 4) {
+                    if (steps == 4) {
                         if (lane == 0) {
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
+                            for (int j = 0; j < APS; ++j) {
                                 tc_cp_scales_if(1u, sf + 4 * j, dsa + 32 * j);
                                 tc_cp_scales_if(1u, sf + 16 + 8 * j, dsb + 32 * j);
                                 tc_cp_scales_if(1u, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                             }
-                            tc_mma_if<MX>(1u, tmem, da, db, sf, sf + 16, acc, IDESC);
 #pragma unroll
-                            for (int j = 1; j < 4; ++j)
-                                tc_mma_if<MX>(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, 1u, IDESC);
+                            for (int j = 0; j < 4; ++j) {
+                                if (MX)
+                                    tc_mma_if<MX>(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1),
+                                                  sf + 16 + 8 * (j >> 1), (acc | (uint32_t)j) ? 1u : 0u,
+                                                  idesc_mx(2u * (uint32_t)(j & 1)));
+                                else
+                                    tc_mma_if<MX>(1u, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
+                                                  (acc | (uint32_t)j) ? 1u : 0u, IDESC);
+                            }
                         }
                         __syncwarp();
                     } else {
-                        for (int j = 0; j < steps; ++j) {
+                        const int atoms = MX ? (steps + 1) / 2 : steps;
+                        for (int j = 0; j < atoms; ++j) {
                             tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
                             tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
                             tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
                         }
-                        for (int j = 0; j < steps; ++j)
-                            tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
-                                          (acc | (uint32_t)j) ? 1u : 0u, IDESC);
+                        for (int j = 0; j < steps; ++j) {
+                            if (MX)
+                                tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1),
+                                              sf + 16 + 8 * (j >> 1), (acc | (uint32_t)j) ? 1u : 0u,
+                                              idesc_mx(2u * (uint32_t)(j & 1)));
+                            else
+                                tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j,
+                                              (acc | (uint32_t)j) ? 1u : 0u, IDESC);
+                        }
                     }
                     acc = 1;
                     tc_commit_pair_if(issue, bar_empty + 8 * s);
@@ -482,9 +562,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (rank == 0) {
             // ---------------- waiter (leader only) ----------------
             // Waits on the accumulator-free and stage-full barriers in the order the
-            // MMA warp consumes them and relays each through a named barrier.  After
-            // a timeout inside a tile it keeps relaying without waiting until the
-            // tile ends, then both warps stop.
+            // MMA warp consumes them and relays each
+            // through a named barrier.  After a timeout inside a tile it keeps
+            // relaying without waiting until the tile ends, then both warps stop.
             // Both warps take the same named barriers in the same order (bar.sync on
             // both sides: neither can run ahead), and leave the tile loop together:
             // the stop decision is written before the per-tile barrier and read by
@@ -508,13 +588,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
-    } else {
+    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // ---------------- epilogue (both CTAs) ----------------
         // Warp w reads TMEM lane quarter w % 4 (the quarter a warp may access) and
-        // columns [128 h, 128 h + 128) of the accumulator, h = (w - 2) / 4.
+        // columns [128 h, 128 h + 128) of the accumulator, h = (w - 2) / 4; row
+        // 32 (w % 4) + lane of this CTA's 128 is the thread's.
+        const int ew = warp - EPI_WARP0;
         const uint32_t q = warp & 3;
-        const int h = (warp - 2) >> 2;
-        const uint32_t tbase = tmem + ((q * 32u) << 16) + 128u * (uint32_t)h;
+        const int hh = ew >> 2;
+        const uint32_t tbase = tmem + ((q * 32u) << 16) + 128u * (uint32_t)hh;
+        const uint32_t stg = smem_base + STAGING_OFF + (uint32_t)ew * CHUNK_BYTES;
+        const uint32_t ep_bar = bar_epi + 8 * ew;
+        uint32_t ep_phase = 0;
         uint64_t policy;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
         const float scale = MX ? 1.0f : __fmul_rn(*p.tsa, *p.tsb);  // MXFP4 has no tensor scale
@@ -527,150 +612,102 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tc_fence_after();
             int mt, nt;
             tile_coords(p, t, mt, nt);
-            const int row = mt * BM + 128 * (int)rank + (int)q * 32 + lane;
-            const bool row_ok = row < p.M;
-            const int c0 = nt * BN + 128 * h;  // first column of this warp's half
-            if (c0 + 128 <= p.N) {
-                // The warp's whole half-row fits in registers: read all of it, hand
-                // TMEM back, then scale and store.
-                if (p.c_bf16) {
-                    uint32_t w[64];
+            const int row0 = mt * BM + 128 * (int)rank + (int)q * 32;  // this warp's 32 rows
+            const int col0 = nt * BN + 128 * hh;                        // and 128 columns
+            const bool rows_in = row0 < p.M;
+            if (p.c_bf16) {
+                // Both 64-column chunks in registers (packed bf16), TMEM handed back,
+                // then each chunk goes out through the staging buffer.
+                uint32_t w[2][32];
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
+                for (int c = 0; c < 2; ++c) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
                         uint32_t r[32];
-                        tmem_ld32(tbase + ch * 32, r);
+                        tmem_ld32(tbase + 64 * c + 32 * half, r);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
-                            const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
-                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[ch * 16 + j]) : "f"(hi), "f"(lo));
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            w[c][16 * half + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), scale),
+                                                              __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
-                    if (!row_ok) continue;
-                    uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + c0;
-                    if (p.epi != GEMM_EPI_PLAIN) {
-                        // Squared ReLU (or its derivative) of the bf16 result, stored, with
-                        // the running max |out| and max |H16 D out| down the 16-row groups
-                        // (lanes 0-15 and 16-31 hold consecutive rows): the butterfly runs
-                        // across lanes, lower lane a + b, upper lane a - b, strides 1..8.
-                        uint16_t *aux = static_cast<uint16_t *>(p.aux) + (int64_t)row * p.ldc + c0;
-                        const bool fwd = p.epi == GEMM_EPI_RELU2_FWD;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            uint32_t o[4];
-                            if (fwd) {
-                                st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
-#pragma unroll
-                                for (int k = 0; k < 4; ++k) o[k] = relu2_pair(w[4 * j + k]);
-                                st_global_v4(aux + 8 * j, o[0], o[1], o[2], o[3], policy);
-                            } else {
-                                const uint4 y = *reinterpret_cast<const uint4 *>(aux + 8 * j);
-                                o[0] = drelu2_pair(w[4 * j], y.x);
-                                o[1] = drelu2_pair(w[4 * j + 1], y.y);
-                                o[2] = drelu2_pair(w[4 * j + 2], y.z);
-                                o[3] = drelu2_pair(w[4 * j + 3], y.w);
-                                st_global_v4(dst + 8 * j, o[0], o[1], o[2], o[3], policy);
-                            }
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                float v = (k & 1) ? bf16hi(o[k >> 1]) : bf16lo(o[k >> 1]);
-                                epi_m0 = fmaxf(epi_m0, fabsf(v));
-                                v = __uint_as_float(__float_as_uint(v) ^ row_sign);
-#pragma unroll
-                                for (int hs = 1; hs < 16; hs <<= 1) {
-                                    const float pv = __shfl_xor_sync(0xFFFFFFFFu, v, hs);
-                                    v = (lane & hs) ? __fsub_rn(pv, v) : __fadd_rn(v, pv);
-                                }
-                                epi_m1 = fmaxf(epi_m1, fabsf(v));
-                            }
-                        }
-                        continue;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
-                } else {
-                    uint32_t v[128];
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t r[32];
-                        tmem_ld32(tbase + ch * 32, r);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[ch * 32 + j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), scale));
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
-                    if (!row_ok) continue;
-                    float *dst = static_cast<float *>(p.C) + (int64_t)row * p.ldc + c0;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) st_global_v4(dst + 4 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3], policy);
                 }
-                continue;
-            }
-            // Ragged right edge: 32 columns at a time, TMEM released after the last read.
-#pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tbase + ch * 32, r);
-                if (ch == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
-                }
-                const int col0 = c0 + ch * 32;
-                if (!row_ok || col0 >= p.N) continue;
-                if (p.c_bf16) {
-                    uint16_t *dst = static_cast<uint16_t *>(p.C) + (int64_t)row * p.ldc + col0;
-                    uint32_t w[16];
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float lo = __fmul_rn(__uint_as_float(r[2 * j]), scale);
-                        const float hi = __fmul_rn(__uint_as_float(r[2 * j + 1]), scale);
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[j]) : "f"(hi), "f"(lo));
-                    }
-                    if (col0 + 32 <= p.N) {
+                for (int c = 0; c < 2; ++c) {
+                    const int x = col0 + 64 * c;
+                    const bool in = rows_in && x < p.N;
+                    if (p.epi == GEMM_EPI_PLAIN) {
+                        store_chunk(&map_c, stg, w[c], lane, x, row0, in);
+                    } else if (p.epi == GEMM_EPI_RELU2_FWD) {
+                        // y, then h = relu(y)^2 with its two amaxes
+                        store_chunk(&map_c, stg, w[c], lane, x, row0, in);
+                        uint32_t o[32];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) st_global_v4(dst + 8 * j, w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3], policy);
+                        for (int k = 0; k < 32; ++k) {
+                            o[k] = relu2_pair(w[c][k]);
+                            amax_pair_rht(o[k], row_sign, lane, epi_m0, epi_m1);
+                        }
+                        store_chunk(&map_aux, stg, o, lane, x, row0, in);
                     } else {
+                        // dY = dh * 2 relu(Y): the forward's Y chunk comes in through the
+                        // staging buffer (TMA load), dY leaves through it
+                        if (lane == 0) {
+                            bulk_wait_read_all();
+                            mbar_expect_tx(ep_bar, CHUNK_BYTES);
+                            tma_load_own(stg, &map_aux, ep_bar, x, row0, policy);
+                        }
+                        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(ep_bar, ep_phase, abort_flag));
+                        ep_phase ^= 1;
+                        uint32_t o[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) dst[j] = (uint16_t)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu));
+                        for (int u = 0; u < 8; ++u) {
+                            const uint4 y = ld_shared_v4(stg + chunk_off(lane, u));
+                            o[4 * u] = drelu2_pair(w[c][4 * u], y.x);
+                            o[4 * u + 1] = drelu2_pair(w[c][4 * u + 1], y.y);
+                            o[4 * u + 2] = drelu2_pair(w[c][4 * u + 2], y.z);
+                            o[4 * u + 3] = drelu2_pair(w[c][4 * u + 3], y.w);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) amax_pair_rht(o[k], row_sign, lane, epi_m0, epi_m1);
+                        store_chunk(&map_c, stg, o, lane, x, row0, in && got);
                     }
-                } else {
-                    float *dst = static_cast<float *>(p.C) + (int64_t)row * p.ldc + col0;
+                }
+            } else {
+                // f32: four 32-column chunks; TMEM handed back after the last read
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + 32 * c, r);
+                    if (c == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), scale));
-                    if (col0 + 32 <= p.N) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) st_global_v4(dst + 4 * j, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3], policy);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) dst[j] = __uint_as_float(r[j]);
-                    }
+                    const int x = col0 + 32 * c;
+                    store_chunk(&map_c, stg, r, lane, x, row0, rows_in && x < p.N);
                 }
             }
         }
+        if (lane == 0) bulk_wait_all();  // every store of this warp complete before the CTA exits
     }
 
-    if (p.epi != GEMM_EPI_PLAIN && warp >= 2 && warp < 2 + EPI_WARPS) {
+    if (p.epi != GEMM_EPI_PLAIN && warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // this CTA's partials of the fused amax: warps, then the 8 epilogue warps
-        float *red = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 128);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             epi_m0 = fmaxf(epi_m0, __shfl_xor_sync(0xFFFFFFFFu, epi_m0, o));
             epi_m1 = fmaxf(epi_m1, __shfl_xor_sync(0xFFFFFFFFu, epi_m1, o));
         }
         if (lane == 0) {
-            red[warp - 2] = epi_m0;
-            red[EPI_WARPS + warp - 2] = epi_m1;
+            red[warp - EPI_WARP0] = epi_m0;
+            red[EPI_WARPS + warp - EPI_WARP0] = epi_m1;
         }
         asm volatile("bar.sync %0, %1;" ::"r"(NB_EPI), "r"(32 * EPI_WARPS) : "memory");
-        if (warp == 2 && lane == 0) {
+        if (warp == EPI_WARP0 && lane == 0) {
             float a = 0.0f, b = 0.0f;
             for (int i = 0; i < EPI_WARPS; ++i) {
                 a = fmaxf(a, red[i]);
@@ -684,7 +721,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
     }
@@ -732,14 +769,36 @@ bool make_scale_map(CUtensorMap *map, const uint8_t *scales, int64_t rows, int64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A row-major [rows x cols] output (or the fused epilogue's bf16 companion)
+// with leading dimension ld elements: box = 128 bytes x 32 rows, 128B swizzle
+// (the epilogue's staging chunk).
+bool make_out_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld, bool bf16) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const uint32_t esz = bf16 ? 2u : 4u;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * esz};
+    cuuint32_t box[2] = {128u / esz, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool MX>
 cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
     const int kbs = MX ? (int)((a.K + 127) / 128) : (int)(a.K / 64);
-    CUtensorMap map_a, map_b, map_sfa, map_sfb;
+    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_c, map_aux;
     if (!make_codes_map(&map_a, a.a_codes, a.M, a.K) || !make_codes_map(&map_b, a.b_codes, a.N, a.K) ||
         !make_scale_map(&map_sfa, a.a_scales, a.M, kbs, kAtomsPerStage<MX>) ||
-        !make_scale_map(&map_sfb, a.b_scales, a.N, kbs, kAtomsPerStage<MX>))
+        !make_scale_map(&map_sfb, a.b_scales, a.N, kbs, kAtomsPerStage<MX>) ||
+        !make_out_map(&map_c, a.C, a.M, a.N, a.ldc, a.c_bf16))
         return cudaErrorInvalidValue;
+    if (a.epi != GEMM_EPI_PLAIN) {
+        if (!make_out_map(&map_aux, a.aux, a.M, a.N, a.ldc, true)) return cudaErrorInvalidValue;
+    } else {
+        map_aux = map_c;  // unused
+    }
     constexpr int kMaxDev = 64;
     static int max_clusters[kMaxDev] = {};
     int dev = 0;
@@ -764,8 +823,6 @@ cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
     KParams p;
     p.tsa = a.a_ts;
     p.tsb = a.b_ts;
-    p.C = a.C;
-    p.ldc = a.ldc;
     p.M = (int)a.M;
     p.N = (int)a.N;
     p.K = (int)a.K;
@@ -778,11 +835,10 @@ cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
     p.num_tiles = p.tiles_m * p.tiles_n;
     p.status = a.status;
     p.epi = a.epi;
-    p.aux = a.aux;
     p.seed = a.seed;
     p.partials = a.partials;
     const int pairs = std::min(p.num_tiles, max_clusters[dev]);
-    gemm_nvfp4_kernel<MX><<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, p);
+    gemm_nvfp4_kernel<MX><<<2 * pairs, THREADS, SMEM_BYTES, s>>>(map_a, map_b, map_sfa, map_sfb, map_c, map_aux, p);
     ++*launches;
     if (a.epi != GEMM_EPI_PLAIN) {
         e = cudaGetLastError();
