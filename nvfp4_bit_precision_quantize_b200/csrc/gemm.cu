@@ -271,6 +271,17 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
     if (__all_sync(0xFFFFFFFFu, try_wait_scoped<CLUSTER>(bar, parity))) return true;
     return mbar_wait_warp_slow<CLUSTER>(bar, parity, abort_flag, honour_abort, limit_ns);
 }
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -562,13 +573,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (rank == 0) {
             // ---------------- waiter (leader only) ----------------
             // Waits on the accumulator-free and stage-full barriers in the order the
-            // MMA warp consumes them and relays each
-            // through a named barrier.  After a timeout inside a tile it keeps
-            // relaying without waiting until the tile ends, then both warps stop.
+            // MMA warp consumes them and relays each through a named barrier.  After
+            // a timeout inside a tile it keeps relaying without waiting until the
+            // tile ends, then both warps stop.
             // Both warps take the same named barriers in the same order (bar.sync on
             // both sides: neither can run ahead), and leave the tile loop together:
             // the stop decision is written before the per-tile barrier and read by
-            // the MMA warp after it.
+            // the MMA warp after it.  (A relay with bar.arrive on the waiter's side,
+            // letting it run ahead, measured no faster: the MMA warp's own issue of
+            // each stage's scale copies and MMAs is the slower party.)
             uint32_t s = 0, ph = 0;
             int tile_i = 0;
             bool ok = true;
@@ -616,24 +629,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int col0 = nt * BN + 128 * hh;                        // and 128 columns
             const bool rows_in = row0 < p.M;
             if (p.c_bf16) {
-                // Both 64-column chunks in registers (packed bf16), TMEM handed back,
-                // then each chunk goes out through the staging buffer.
+                // All 128 accumulator columns into registers, TMEM handed back, then
+                // scaled and packed to bf16, each 64-column chunk out through the
+                // staging buffer.
                 uint32_t w[2][32];
+                {
+                    uint32_t r[4][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                    for (int k = 0; k < 4; ++k) tmem_ld32_nowait(tbase + 32 * k, r[k]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t r[32];
-                        tmem_ld32(tbase + 64 * c + 32 * half, r);
+                    for (int k = 0; k < 4; ++k)
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            w[c][16 * half + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * j]), scale),
-                                                              __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
-                    }
+                            w[k >> 1][16 * (k & 1) + j] = pack_bf16x2(__fmul_rn(__uint_as_float(r[k][2 * j]), scale),
+                                                                      __fmul_rn(__uint_as_float(r[k][2 * j + 1]), scale));
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const int x = col0 + 64 * c;

@@ -771,7 +771,7 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
     QParams p{a.x, a.R, a.C, a.ld, a.seed, a.amax_in, a.partials, num_partials, a.codes, a.scales,
               a.tensor_scale};
     p.aligned32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && ((a.ld * (int64_t)sizeof(T)) % 32 == 0);
-    constexpr int N = Vec<T>::N;
+    constexpr int N = Vec<T>::N;  // columns per lane of the colwise kernels
     if (!a.colwise) {
         constexpr int tile_r = sizeof(T) == 2 ? 32 : 16;  // rows per tile of quantize_rowwise_kernel
         const int64_t tiles = ((a.C / 16 + 31) / 32) * ((a.R + 127) / 128) * (128 / tile_r);
