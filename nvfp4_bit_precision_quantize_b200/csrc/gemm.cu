@@ -17,12 +17,19 @@
 //                      (128-byte swizzle) and scale atoms (A: its 128 rows;
 //                      B: all 256 rows) into a 5-stage ring; completion bytes
 //                      of both CTAs are counted on the leader's barrier;
-//   warp 1             allocates TMEM (pair-wide); on the leader the whole
-//                      warp runs the issue loop and one lane, by predicate,
-//                      copies each stage's scales into TMEM (tcgen05.cp,
-//                      cta_group::2) and issues the MMAs; tcgen05.commit
-//                      multicast to both CTAs frees the stage;
-//   warp 10            waiter (leader): polls the stage-full and
+//   warp 1             allocates TMEM (pair-wide); on the leader one lane issues
+//                      the MMAs, four per 256-k stage, reading the stage's
+//                      scales from its TMEM slot; tcgen05.commit multicast to
+//                      both CTAs frees the stage;
+//   warps 11-12        scale copiers (leader), alternate stages: once a stage
+//                      has landed, copy its scale atoms into the stage's TMEM
+//                      slot (tcgen05.cp, cta_group::2) and commit to the
+//                      stage's scale barrier.  Issued from their own warps,
+//                      the copies (twelve per stage) overlap the MMAs of
+//                      earlier stages instead of queueing in front of them:
+//                      moving them out of the MMA warp took the 8192 x 20480
+//                      x 5120 GEMM from 0.53 to 0.37 ms;
+//   warp 10            waiter (leader): polls the stage-scale and
 //                      accumulator-free barriers and relays each event to the
 //                      MMA warp through a hardware named barrier, so that the
 //                      issuing warp never waits on shared memory;
@@ -37,7 +44,7 @@
 // per-stage TMEM slots, keeping the MMA warp's pipe free of copies) were
 // measured slower: the extra hop on every stage's refill path cost more than
 // the ~24 tensor-pipe cycles per copy it saves, with five stages in flight.
-// TMEM: accumulator columns [0, 256), then the 48 scale columns of one stage.
+// TMEM: accumulator columns [0, 256), then one 48-column scale slot per stage.
 // Tiles are visited in groups of 8 tile columns so that the pairs running at
 // the same time share A and B panels in L2.  Every mbarrier wait is bounded
 // (about 2 s of %globaltimer); on expiry the CTA records
@@ -70,14 +77,17 @@ constexpr int BAR_OFF = STAGING_OFF + EPI_WARPS * CHUNK_BYTES;
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-constexpr int THREADS = 352;                    // producer, MMA, 8 epilogue warps, waiter
-constexpr int MMA_WARP = 1, EPI_WARP0 = 2, WAITER_WARP = 10;
+constexpr int SF_WARPS = 2;                     // scale copiers, taking alternate k-stages
+constexpr int THREADS = 32 * (11 + SF_WARPS);   // producer, MMA, 8 epilogue warps, waiter, copiers
+constexpr int MMA_WARP = 1, EPI_WARP0 = 2, WAITER_WARP = 10, SF_WARP0 = 11;
 // Hardware named barriers (64 threads: the waiter warp and the MMA warp).
 constexpr uint32_t NB_ACC = 1;     // accumulator free for the next tile
 constexpr uint32_t NB_STAGE0 = 2;  // NB_STAGE0 + s: stage s loaded
 constexpr uint32_t NB_EPI = NB_STAGE0 + STAGES;  // the 8 epilogue warps (fused amax reduction)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_SF = 256;              // SFA 4 x 4 columns, then SFB 4 x 8 columns
+constexpr uint32_t TMEM_SF = 256;              // scale slot of stage s at TMEM_SF + 48 s
+constexpr uint32_t SF_SLOT_COLS = 48;          // SFA 4 x 4 columns, then SFB 4 x 8 columns
+static_assert(TMEM_SF + STAGES * SF_SLOT_COLS <= TMEM_COLS, "TMEM columns");
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 20000000ull;
 constexpr int kTimeoutStatus = 7;              // NVFP4_ERR_DEVICE_TIMEOUT
@@ -412,7 +422,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t bar_acce = smem_u32(bars + 2 * STAGES + 1);   // leader: accumulator read (16 epilogue warps)
     const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2);  // leader: every MMA done
     const uint32_t bar_epi = smem_u32(bars + 2 * STAGES + 3);    // [8] each CTA: an epilogue warp's aux chunk
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3 + EPI_WARPS);
+    const uint32_t bar_sf = smem_u32(bars + 2 * STAGES + 3 + EPI_WARPS);          // [S] leader: stage's scales in TMEM
+    const uint32_t bar_sf_drain = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS);    // [2] leader: a copier's copies done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 3 + EPI_WARPS + SF_WARPS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *stop_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // waiter -> MMA warp, per tile
     float *red = reinterpret_cast<float *>(tmem_slot + 4);                      // fused amax: 2 x 8 warps
@@ -426,7 +438,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_sf + 8 * s, 1);
         }
+        for (int c = 0; c < SF_WARPS; ++c) mbar_init(bar_sf_drain + 8 * c, 1);
         mbar_init(bar_accf, 1);
         mbar_init(bar_acce, 2 * EPI_WARPS);
         mbar_init(bar_drain, 1);
@@ -502,26 +516,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 uint32_t acc = 0;  // the first MMA of a tile overwrites the accumulator
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    // Stage s has landed (the waiter saw its barrier complete).
+                    // Stage s has landed and its scales are in TMEM slot s (the waiter saw
+                    // the scale copier's barrier complete).
                     named_sync(NB_STAGE0 + s);
+                    tc_fence_after();
                     const uint32_t sa = smem_base + s * STAGE_BYTES;
                     const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + A_BYTES);
-                    const uint64_t dsa = sdesc_scales(sa + SF_OFF);
-                    const uint64_t dsb = sdesc_scales(sa + SF_OFF + SFA_BYTES);
-                    const uint32_t sf = tmem + TMEM_SF;
-                    // Descriptor addresses are in 16-byte units: +32 per 512-byte atom,
-                    // +128 for B's second 128-row tile, +2 per 64-k step of codes.
+                    const uint32_t sf = tmem + TMEM_SF + SF_SLOT_COLS * s;
+                    // Descriptor addresses are in 16-byte units: +2 per 64-k step of codes.
                     // Scales: A atom j at sf + 4 j, B atoms at sf + 16 + 8 j (rows 0-127)
                     // and sf + 20 + 8 j (rows 128-255); MXFP4 atom j serves steps 2j, 2j+1.
                     const int steps = kt < kfull ? 4 : ktail;
                     if (steps == 4) {
                         if (lane == 0) {
-#pragma unroll
-                            for (int j = 0; j < APS; ++j) {
-                                tc_cp_scales_if(1u, sf + 4 * j, dsa + 32 * j);
-                                tc_cp_scales_if(1u, sf + 16 + 8 * j, dsb + 32 * j);
-                                tc_cp_scales_if(1u, sf + 20 + 8 * j, dsb + 128 + 32 * j);
-                            }
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 if (MX)
@@ -535,12 +542,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         }
                         __syncwarp();
                     } else {
-                        const int atoms = MX ? (steps + 1) / 2 : steps;
-                        for (int j = 0; j < atoms; ++j) {
-                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
-                        }
                         for (int j = 0; j < steps; ++j) {
                             if (MX)
                                 tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1),
@@ -572,8 +573,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp == WAITER_WARP) {
         if (rank == 0) {
             // ---------------- waiter (leader only) ----------------
-            // Waits on the accumulator-free and stage-full barriers in the order the
-            // MMA warp consumes them and relays each through a named barrier.  After
+            // Waits on the accumulator-free barrier and on each stage's scale barrier
+            // (the copier signals it after the stage landed and its scales reached
+            // TMEM) in the order the MMA warp consumes them and relays each through
+            // a named barrier.  After
             // a timeout inside a tile it keeps relaying without waiting until the
             // tile ends, then both warps stop.
             // Both warps take the same named barriers in the same order (bar.sync on
@@ -592,7 +595,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 named_sync(NB_ACC);
                 if (stop) break;
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    if (ok) ok = mbar_wait_warp(bar_full + 8 * s, ph, abort_flag);
+                    if (ok) ok = mbar_wait_warp(bar_sf + 8 * s, ph, abort_flag);
                     named_sync(NB_STAGE0 + s);
                     if (++s == STAGES) {
                         s = 0;
@@ -600,6 +603,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                 }
             }
+        }
+    } else if (warp >= SF_WARP0 && warp < SF_WARP0 + SF_WARPS) {
+        if (rank == 0) {
+            // ---------------- scale copiers (leader's warps 11-12, lane 0 issues) ----------------
+            // Copier c takes the k-stages i with i % 2 == c: once stage s has landed,
+            // its scale atoms go into TMEM slot s (tcgen05.cp, both CTAs), then a
+            // commit arrives on bar_sf[s] when the copies are done.  A copy occupies
+            // its issuing warp for ~70 cycles, so one warp alone needs ~850 cycles per
+            // stage, against 512 for the stage's four MMAs; two warps keep ahead of
+            // the MMA warp.  Slot s is free again once stage s has landed anew: the
+            // producer refills the stage only after the MMAs that read the slot have
+            // completed.
+            const int mine = warp - SF_WARP0;
+            const uint32_t issue = lane == 0 ? 1u : 0u;
+            uint32_t s = 0, ph = 0;
+            bool ok = true;
+            int it = 0;
+            for (int t = cid; t < p.num_tiles && ok; t += ncl) {
+                for (int kt = 0; kt < num_kt; ++kt, ++it) {
+                    if (it % SF_WARPS == mine) {
+                        if (!mbar_wait_warp(bar_full + 8 * s, ph, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sa = smem_base + s * STAGE_BYTES;
+                        const uint64_t dsa = sdesc_scales(sa + SF_OFF);
+                        const uint64_t dsb = sdesc_scales(sa + SF_OFF + SFA_BYTES);
+                        const uint32_t sf = tmem + TMEM_SF + SF_SLOT_COLS * s;
+                        // Descriptor addresses in 16-byte units: +32 per 512-byte atom,
+                        // +128 for B's second 128-row tile.
+                        const int steps = kt < p.kfull ? 4 : p.ktail;
+                        const int atoms = MX ? (steps + 1) / 2 : steps;
+                        for (int j = 0; j < atoms; ++j) {
+                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
+                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
+                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
+                        }
+                        tc_commit_self_if(issue, bar_sf + 8 * s);
+                    }
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            tc_commit_self_if(issue, bar_sf_drain + 8 * mine);
+            mbar_wait_warp(bar_sf_drain + 8 * mine, 0, abort_flag, false);  // every copy done before TMEM is freed
         }
     } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // ---------------- epilogue (both CTAs) ----------------
