@@ -261,7 +261,69 @@ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t b, int64_t KB
 // 16-point random Hadamard transform in registers: sign flips (xor of the sign
 // bit), the fixed-order butterfly over strides 1, 2, 4, 8, then a 1/4 scale.
 // ---------------------------------------------------------------------------
-// The fixed-order butterfly alone (strides 1, 2, 4, 8), unnormalised: z = H16 v.
+// ---------------------------------------------------------------------------
+// Packed binary32 pairs: the f32x2 add / sub / mul of sm_100 round each half
+// exactly as the scalar operation does, so a pair operation gives the same
+// bits as two scalar ones, in one instruction.  Halves live in one 64-bit
+// register pair (low half = first element).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ float f2lo(uint64_t d) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+    return lo;
+}
+__device__ __forceinline__ float f2hi(uint64_t d) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+    return hi;
+}
+__device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2_ru(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rp.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2_rn(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2_rn(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The fixed-order butterfly alone (strides 1, 2, 4, 8), unnormalised: z = H16 v,
+// with its outputs as pairs p[k] = (z[2k], z[2k+1]).  Stride 1 runs on scalars
+// and writes straight into the pairs; strides 2, 4 and 8 pair element i with
+// i + h for both halves at once (pair stride h / 2).  The operations and their
+// order are those of the scalar butterfly.
+__device__ __forceinline__ void fwht16_x2(const float *v, uint64_t (&p)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) p[k] = f2(__fadd_rn(v[2 * k], v[2 * k + 1]), __fsub_rn(v[2 * k], v[2 * k + 1]));
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k & h) continue;
+            const uint64_t a = p[k], b = p[k + h];
+            p[k] = add2_rn(a, b);
+            p[k + h] = sub2_rn(a, b);
+        }
+    }
+}
+// The same butterfly on scalars (for callers that only need max |z|: fewer
+// register-pair constraints than the packed form).
 __device__ __forceinline__ void fwht16(float *v) {
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {

@@ -16,21 +16,23 @@
 //   warp 0 (one lane)  producer: TMA loads of this CTA's A and B code tiles
 //                      (128-byte swizzle) and scale atoms (A: its 128 rows;
 //                      B: all 256 rows) into a 5-stage ring; completion bytes
-//                      of both CTAs are counted on the leader's barrier;
+//                      of both CTAs are counted on the leader's barriers, the
+//                      scale atoms on a barrier of their own;
 //   warp 1             allocates TMEM (pair-wide); on the leader one lane issues
 //                      the MMAs, four per 256-k stage, reading the stage's
 //                      scales from its TMEM slot; tcgen05.commit multicast to
 //                      both CTAs frees the stage;
-//   warps 11-12        scale copiers (leader), alternate stages: once a stage
-//                      has landed, copy its scale atoms into the stage's TMEM
+//   warps 11-12        scale copiers (leader), alternate stages: once a stage's
+//                      scale atoms have landed, copy them into the stage's TMEM
 //                      slot (tcgen05.cp, cta_group::2) and commit to the
 //                      stage's scale barrier.  Issued from their own warps,
 //                      the copies (twelve per stage) overlap the MMAs of
 //                      earlier stages instead of queueing in front of them:
 //                      moving them out of the MMA warp took the 8192 x 20480
 //                      x 5120 GEMM from 0.53 to 0.37 ms;
-//   warp 10            waiter (leader): polls the stage-scale and
-//                      accumulator-free barriers and relays each event to the
+//   warp 10            waiter (leader): polls the stage's code and scale-copy
+//                      barriers and the accumulator-free barrier, and relays
+//                      each event to the
 //                      MMA warp through a hardware named barrier, so that the
 //                      issuing warp never waits on shared memory;
 //   warps 2..9         epilogue: two warps per 32-lane TMEM quarter, each
@@ -424,7 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t bar_epi = smem_u32(bars + 2 * STAGES + 3);    // [8] each CTA: an epilogue warp's aux chunk
     const uint32_t bar_sf = smem_u32(bars + 2 * STAGES + 3 + EPI_WARPS);          // [S] leader: stage's scales in TMEM
     const uint32_t bar_sf_drain = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS);    // [2] leader: a copier's copies done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 3 + EPI_WARPS + SF_WARPS);
+    const uint32_t bar_sfull = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS + SF_WARPS);  // [S] leader: scale bytes
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 3 + EPI_WARPS + SF_WARPS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *stop_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // waiter -> MMA warp, per tile
     float *red = reinterpret_cast<float *>(tmem_slot + 4);                      // fused amax: 2 x 8 warps
@@ -439,6 +442,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
             mbar_init(bar_sf + 8 * s, 1);
+            mbar_init(bar_sfull + 8 * s, 1);
         }
         for (int c = 0; c < SF_WARPS; ++c) mbar_init(bar_sf_drain + 8 * c, 1);
         mbar_init(bar_accf, 1);
@@ -471,7 +475,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
             uint32_t s = 0, ph = 0;
             bool ok = true;
-            constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + 3 * APS * 512;  // bytes per CTA per stage
+            // Bytes per CTA per stage: the scale atoms complete on their own barrier, so
+            // that the copiers can move them into TMEM while the codes still land.
+            constexpr uint32_t CODES_TX = A_BYTES + B_BYTES, SCALES_TX = 3 * APS * 512;
             for (int t = cid; t < p.num_tiles && ok; t += ncl) {
                 int mt, nt;
                 tile_coords(p, t, mt, nt);
@@ -484,15 +490,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     const uint32_t st = smem_base + s * STAGE_BYTES;
                     const uint32_t full_leader = mapa(bar_full + 8 * s, 0);
+                    const uint32_t sfull_leader = mapa(bar_sfull + 8 * s, 0);
                     // Out-of-range rows, columns and atoms are zero-filled and still
-                    // counted, so every stage brings exactly STAGE_TX bytes per CTA.
-                    if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * STAGE_TX);
+                    // counted, so every stage brings exactly CODES_TX + SCALES_TX bytes
+                    // per CTA.
+                    if (rank == 0) {
+                        mbar_expect_tx(bar_sfull + 8 * s, 2 * SCALES_TX);
+                        mbar_expect_tx(bar_full + 8 * s, 2 * CODES_TX);
+                    }
+                    tma_load_pair(st + SF_OFF, &map_sfa, sfull_leader, 0, ya + kt * APS, policy);
+                    tma_load_pair(st + SF_OFF + SFA_BYTES, &map_sfb, sfull_leader, 0, yb + kt * APS, policy);
+                    tma_load_pair(st + SF_OFF + SFA_BYTES + 2048, &map_sfb, sfull_leader, 0, yb + p.kbs + kt * APS,
+                                  policy);
                     tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
                     tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
-                    tma_load_pair(st + SF_OFF, &map_sfa, full_leader, 0, ya + kt * APS, policy);
-                    tma_load_pair(st + SF_OFF + SFA_BYTES, &map_sfb, full_leader, 0, yb + kt * APS, policy);
-                    tma_load_pair(st + SF_OFF + SFA_BYTES + 2048, &map_sfb, full_leader, 0, yb + p.kbs + kt * APS,
-                                  policy);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
@@ -566,25 +577,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_wait_warp(bar_drain, 0, abort_flag, false);
             if (*abort_flag) {
                 // Stages the producers may still be filling: wait (briefly) for their bytes.
-                for (int k = consumed; k < consumed + STAGES; ++k)
+                for (int k = consumed; k < consumed + STAGES; ++k) {
                     mbar_wait_warp(bar_full + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
+                    mbar_wait_warp(bar_sfull + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false,
+                                   DRAIN_LIMIT_NS);
+                }
             }
         }
     } else if (warp == WAITER_WARP) {
         if (rank == 0) {
             // ---------------- waiter (leader only) ----------------
-            // Waits on the accumulator-free barrier and on each stage's scale barrier
-            // (the copier signals it after the stage landed and its scales reached
-            // TMEM) in the order the MMA warp consumes them and relays each through
-            // a named barrier.  After
+            // Waits on the accumulator-free barrier and, per stage, on its code bytes
+            // and on its scale barrier (a copier signals it once the stage's scale
+            // atoms reached TMEM) in the order the MMA warp consumes them, and relays
+            // each through a named barrier.  After
             // a timeout inside a tile it keeps relaying without waiting until the
             // tile ends, then both warps stop.
             // Both warps take the same named barriers in the same order (bar.sync on
             // both sides: neither can run ahead), and leave the tile loop together:
             // the stop decision is written before the per-tile barrier and read by
-            // the MMA warp after it.  (A relay with bar.arrive on the waiter's side,
-            // letting it run ahead, measured no faster: the MMA warp's own issue of
-            // each stage's scale copies and MMAs is the slower party.)
+            // the MMA warp after it.
             uint32_t s = 0, ph = 0;
             int tile_i = 0;
             bool ok = true;
@@ -595,6 +607,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 named_sync(NB_ACC);
                 if (stop) break;
                 for (int kt = 0; kt < num_kt; ++kt) {
+                    if (ok) ok = mbar_wait_warp(bar_full + 8 * s, ph, abort_flag);
                     if (ok) ok = mbar_wait_warp(bar_sf + 8 * s, ph, abort_flag);
                     named_sync(NB_STAGE0 + s);
                     if (++s == STAGES) {
@@ -607,14 +620,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     } else if (warp >= SF_WARP0 && warp < SF_WARP0 + SF_WARPS) {
         if (rank == 0) {
             // ---------------- scale copiers (leader's warps 11-12, lane 0 issues) ----------------
-            // Copier c takes the k-stages i with i % 2 == c: once stage s has landed,
-            // its scale atoms go into TMEM slot s (tcgen05.cp, both CTAs), then a
-            // commit arrives on bar_sf[s] when the copies are done.  A copy occupies
+            // Copier c takes the k-stages i with i % 2 == c: once stage s's scale
+            // atoms have landed (bar_sfull, usually before the code tiles), they go
+            // into TMEM slot s (tcgen05.cp, both CTAs), then a commit arrives on
+            // bar_sf[s] when the copies are done.  A copy occupies
             // its issuing warp for ~70 cycles, so one warp alone needs ~850 cycles per
             // stage, against 512 for the stage's four MMAs; two warps keep ahead of
-            // the MMA warp.  Slot s is free again once stage s has landed anew: the
-            // producer refills the stage only after the MMAs that read the slot have
-            // completed.
+            // the MMA warp.  Slot s is free again once stage s's scales have landed
+            // anew: the producer refills the stage only after the MMAs that read the
+            // slot have completed.
             const int mine = warp - SF_WARP0;
             const uint32_t issue = lane == 0 ? 1u : 0u;
             uint32_t s = 0, ph = 0;
@@ -623,7 +637,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             for (int t = cid; t < p.num_tiles && ok; t += ncl) {
                 for (int kt = 0; kt < num_kt; ++kt, ++it) {
                     if (it % SF_WARPS == mine) {
-                        if (!mbar_wait_warp(bar_full + 8 * s, ph, abort_flag)) {
+                        if (!mbar_wait_warp(bar_sfull + 8 * s, ph, abort_flag)) {
                             ok = false;
                             break;
                         }

@@ -235,16 +235,33 @@ __device__ __forceinline__ uint32_t sr_carry(const uint4 &w, int e) {  // e = id
 }
 
 // 16 E2M1 codes of one block (element 0 in the lowest nibble of .x), from the
-// block's values and element scale; SR draws from w0 (elements 0-7) and w1
-// (8-15).  A block whose inv is 0 encodes +0 everywhere (the products are +-0,
-// and the sign bits are cleared).
+// block's values as pairs p[k] = (v[2k], v[2k+1]) and its element scale; SR
+// draws from w0 (elements 0-7) and w1 (8-15).  A block whose inv is 0 encodes
+// +0 everywhere (the products are +-0, and the sign bits are cleared).  The
+// products and the SR rounding steps run as pair operations (same bits as
+// sr_e2m1_value on each element).
 template <bool SR>
-__device__ __forceinline__ uint2 encode16(const float (&v)[16], float inv, const uint4 &w0, const uint4 &w1) {
+__device__ __forceinline__ uint2 encode16_x2(const uint64_t (&p)[8], float inv, const uint4 &w0, const uint4 &w1) {
+    const uint64_t inv2 = f2(inv, inv);
     float q[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float r = __fmul_rn(v[i], inv);
-        q[i] = SR ? sr_e2m1_value(r, sr_carry(i < 8 ? w0 : w1, i & 7)) : r;
+    for (int k = 0; k < 8; ++k) {
+        const uint64_t r = mul2_rn(p[k], inv2);
+        const float r0 = f2lo(r), r1 = f2hi(r);
+        if (SR) {
+            const float a0 = fminf(fabsf(r0), 7.0f), a1 = fminf(fabsf(r1), 7.0f);
+            const uint64_t base = f2(a0 < 1.0f ? 1.0f : 0.0f, a1 < 1.0f ? 1.0f : 0.0f);
+            const uint64_t t = add2_ru(f2(a0, a1), base);
+            const uint32_t c0 = sr_carry(k < 4 ? w0 : w1, (2 * k) & 7), c1 = sr_carry(k < 4 ? w0 : w1, (2 * k + 1) & 7);
+            const uint64_t up = f2(__uint_as_float((__float_as_uint(f2lo(t)) + c0) & 0xFFC00000u),
+                                   __uint_as_float((__float_as_uint(f2hi(t)) + c1) & 0xFFC00000u));
+            const uint64_t d = sub2_rn(up, base);
+            q[2 * k] = copysignf(f2lo(d), r0);
+            q[2 * k + 1] = copysignf(f2hi(d), r1);
+        } else {
+            q[2 * k] = r0;
+            q[2 * k + 1] = r1;
+        }
     }
     uint2 c = make_uint2(e2m1x8(q), e2m1x8(q + 8));
     if (inv == 0.0f) {
@@ -252,6 +269,13 @@ __device__ __forceinline__ uint2 encode16(const float (&v)[16], float inv, const
         c.y &= 0x77777777u;
     }
     return c;
+}
+template <bool SR>
+__device__ __forceinline__ uint2 encode16(const float (&v)[16], float inv, const uint4 &w0, const uint4 &w1) {
+    uint64_t p[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) p[k] = f2(v[2 * k], v[2 * k + 1]);
+    return encode16_x2<SR>(p, inv, w0, w1);
 }
 
 // Loads of one 16-element block row segment: 8 (bf16) or 16 (f32) words.
@@ -510,29 +534,33 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
             }
             float scale_in;  // the element scale the block's values are multiplied by
             uint32_t sb;
+            uint64_t pv[8];  // the block's values as pairs (v[2k], v[2k+1])
+            float m = 0.0f;
             if (RHT) {
-                fwht16(v);
-                float m = 0.0f;
+                fwht16_x2(v, pv);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+                for (int k = 0; k < 8; ++k) m = fmaxf(m, fmaxf(fabsf(f2lo(pv[k])), fabsf(f2hi(pv[k]))));
                 sb = block_scale_code(__fmul_rn(m, 0.25f), ctx);  // max |z/4| = RN(max|z| / 4)
                 if (fold) {
                     scale_in = s_inv4[sb];
                 } else {
+                    const uint64_t quarter = f2(0.25f, 0.25f);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+                    for (int k = 0; k < 8; ++k) pv[k] = mul2_rn(pv[k], quarter);
                     scale_in = s_inv[sb];
                 }
             } else {
-                float m = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+                for (int k = 0; k < 8; ++k) {
+                    pv[k] = f2(v[2 * k], v[2 * k + 1]);
+                    m = fmaxf(m, fmaxf(fabsf(v[2 * k]), fabsf(v[2 * k + 1])));
+                }
                 sb = block_scale_code(m, ctx);
                 scale_in = s_inv[sb];
             }
             uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
             if (SR) sr_words16((uint64_t)(c + j) * (uint64_t)K + (uint64_t)rg, keys, w0, w1);  // rg % 16 == 0
-            const uint2 code = encode16<SR>(v, scale_in, w0, w1);
+            const uint2 code = encode16_x2<SR>(pv, scale_in, w0, w1);
             {  // this group's 8 code bytes: half h of the lane's 16-byte unit for column j
                 const int qu = j * P + warp;
                 reinterpret_cast<uint2 *>(s_units)[(qu * 32 + (lane ^ (qu & 7))) * 2 + h] = code;
