@@ -589,6 +589,13 @@ def run_profile_case(case):
         q = None
         for _ in range(3):
             q = B.nvfp4_quantize(x, out=q, ws=ws, seed=SEED, **kw)
+    elif case == "quant_h":  # the step's h_c: colwise, RHT, RTN, amax supplied (as the relu^2 epilogue does)
+        x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, FFN)))).to(dev).abs()
+        amax = x.float().abs().max().reshape(1)
+        ws = B.workspace(B.nvfp4_quantize_workspace_size(), dev)
+        q = None
+        for _ in range(3):
+            q = B.nvfp4_quantize(x, orientation=B.NVFP4_COLWISE, rht=True, amax_in=amax, out=q, ws=ws, seed=SEED)
     elif case == "quant_mx":  # MXFP4 rowwise of an h-shaped tensor
         x = W.bits_to_torch_bf16(W.bf16_bits(W.normal(rng, (M_TOK, FFN)))).to(dev)
         q = None
@@ -614,7 +621,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy", "quant_dual", "quant_mx"],
+    ap.add_argument("--profile-case", choices=["gemm", "quant_x", "quant_dy", "quant_dual", "quant_h", "quant_mx"],
                     help="run one kernel a few times for an ncu capture instead of the benchmark")
     args = ap.parse_args()
     if args.profile_case:
