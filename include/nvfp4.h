@@ -359,6 +359,24 @@ NVFP4_API nvfp4_status nvfp4_check(void *workspace, cudaStream_t stream);
 NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_bytes, uint64_t limit_ns,
                                                    cudaStream_t stream);
 
+/* Tensor-pipe rate probe (measurement only; the pages give Blackwell's NVFP4
+ * tensor cores as the engine of the method: nerdman.de, section "Was konkret
+ * passiert ist").  Every CTA pair the device can hold at once issues `iters`
+ * rounds of the GEMM's stage -- four M256 N256 K64 block-scaled MMAs,
+ * kind::mxf4nvf4 block16 (mx = 0) or kind::mxf4 block32 (mx = 1), with the
+ * GEMM's own descriptors -- on operands resident in shared memory and scales
+ * resident in TMEM, and writes the %clock64 cycles from its first MMA to the
+ * completion of its last to cycles[pair] (device memory, cycles_len >= the
+ * number of pairs; *pairs_out, host memory, receives that number).  FLOPs per
+ * pair: iters * 4 * 2 * 256 * 256 * 64.  iters: 1 .. 1000000.  Asynchronous:
+ * time it with events on `stream`; a completion not seen within ~2 s records
+ * NVFP4_ERR_DEVICE_TIMEOUT in the workspace status word (>= 256 bytes,
+ * 16-byte aligned, caller-owned).  Launch errors: NVFP4_ERR_INVALID_ARG (null
+ * pointer, mx not 0/1, iters out of range, cycles_len too small),
+ * NVFP4_ERR_WORKSPACE, NVFP4_ERR_ALIGNMENT, NVFP4_ERR_UNSUPPORTED_DEVICE. */
+NVFP4_API nvfp4_status nvfp4_selftest_mma_rate(int mx, int64_t iters, uint64_t *cycles, int64_t cycles_len,
+                                               int *pairs_out, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* Number of kernel launches the most recent successful call on this host
  * thread issued (launch accounting for benchmarks). */
 NVFP4_API int nvfp4_last_launch_count(void);

@@ -37,7 +37,7 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
            "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
-           "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd")
+           "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd", "nvfp4_selftest_mma_rate")
 
 
 class CTensor(C.Structure):
@@ -84,6 +84,7 @@ def load():
         "nvfp4_status_string": (C.c_char_p, [i32]),
         "nvfp4_linear_fwd_noalloc": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp]),
         "nvfp4_selftest_wait_timeout": (i32, [vp, sz, u64, vp]),
+        "nvfp4_selftest_mma_rate": (i32, [i32, i64, vp, i64, C.POINTER(C.c_int), vp, sz, vp]),
         "nvfp4_quantize_dual_workspace_size": (sz, []),
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
         "nvfp4_relu2_fwd_amax": (i32, [vp, vp, i64, vp, vp, sz, vp]),
@@ -529,6 +530,19 @@ def nvfp4_selftest_wait_timeout(ws, limit_ns, stream=None):
     _on_device(ws)
     _ok(load().nvfp4_selftest_wait_timeout(_ptr(ws), _workspace(ws), int(limit_ns), _stream(stream)),
         "nvfp4_selftest_wait_timeout")
+
+
+def nvfp4_selftest_mma_rate(cycles, ws, iters, mx=False, stream=None):
+    """Launch the tensor-pipe rate probe; `cycles` is an int64 device tensor with at
+    least SMs/2 entries.  Returns the number of CTA pairs that ran (cycles[:pairs]
+    hold their cycle counts once the stream reaches the launch)."""
+    _on_device(cycles, ws)
+    if cycles.dtype != torch.int64 or not cycles.is_contiguous():
+        raise ValueError("cycles must be a contiguous int64 tensor")
+    pairs = C.c_int(0)
+    _ok(load().nvfp4_selftest_mma_rate(1 if mx else 0, int(iters), _ptr(cycles), cycles.numel(), C.byref(pairs),
+                                       _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_selftest_mma_rate")
+    return pairs.value
 
 
 def nvfp4_last_launch_count():

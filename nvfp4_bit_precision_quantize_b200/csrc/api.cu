@@ -602,6 +602,19 @@ nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_bytes, uint6
     return call.done(from_cuda(launch_wait_timeout(static_cast<int *>(workspace), limit_ns, stream, &call.launches)));
 }
 
+nvfp4_status nvfp4_selftest_mma_rate(int mx, int64_t iters, uint64_t *cycles, int64_t cycles_len, int *pairs_out,
+                                     void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    Call call(__func__);
+    if (!cycles || !pairs_out || (mx != 0 && mx != 1) || iters < 1 || iters > 1000000) return NVFP4_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < kStatusBytes) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace) || reinterpret_cast<uintptr_t>(cycles) % 8 != 0) return NVFP4_ERR_ALIGNMENT;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    if (cycles_len < num_sms() / 2) return NVFP4_ERR_INVALID_ARG;
+    return call.done(from_cuda(launch_mma_rate(mx == 1, iters, cycles, cycles_len, pairs_out,
+                                               static_cast<int *>(workspace), stream, &call.launches)));
+}
+
 int nvfp4_last_launch_count(void) { return g_last_launches; }
 
 const char *nvfp4_status_string(nvfp4_status status) {

@@ -927,6 +927,113 @@ cudaError_t launch_gemm_t(const GemmArgs &a, cudaStream_t s, int *launches) {
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-pipe rate probe (measurement only).  Every CTA pair issues `iters`
+// rounds of the GEMM's stage -- four M256 N256 K64 block-scaled MMAs with the
+// same descriptors -- on one stage of operands resident in shared memory (a
+// fixed byte pattern: every byte is a valid pair of E2M1 codes) and scales
+// resident in TMEM (all 1.0), with a commit per round as the GEMM has.  The
+// issuing thread records the %clock64 cycles from its first MMA to the
+// completion of the last.  Shared memory is sized so that one CTA fits per SM.
+// ---------------------------------------------------------------------------
+constexpr int PROBE_THREADS = 128;
+constexpr int PROBE_SMEM = 120 * 1024;  // > half an SM's shared memory: one CTA per SM
+static_assert(STAGE_BYTES + 64 + 1024 <= PROBE_SMEM, "probe shared memory");
+
+template <bool MX>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PROBE_THREADS, 1)
+    mma_rate_kernel(uint64_t *cycles, int64_t iters, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint32_t *words = reinterpret_cast<uint32_t *>(smem);
+    for (int i = threadIdx.x; i < SF_OFF / 4; i += PROBE_THREADS) words[i] = (uint32_t)i * 2654435761u;
+    for (int i = threadIdx.x; i < (SFA_BYTES + SFB_BYTES) / 4; i += PROBE_THREADS)
+        words[SF_OFF / 4 + i] = MX ? 0x7F7F7F7Fu : 0x38383838u;  // E8M0 / E4M3 encodings of 1.0
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGE_BYTES);
+    const uint32_t bar_round = smem_u32(bars), bar_drain = smem_u32(bars + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 3);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cta_rank();
+    if (threadIdx.x == 0) {
+        mbar_init(bar_round, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    fence_proxy_async();  // the operand bytes, written by threads, are read by the tensor cores
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (rank == 0 && warp == 0) {
+        const uint32_t issue = lane == 0 ? 1u : 0u;
+        const uint32_t sa = smem_u32(smem);
+        const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + A_BYTES);
+        const uint64_t dsa = sdesc_scales(sa + SF_OFF), dsb = sdesc_scales(sa + SF_OFF + SFA_BYTES);
+        const uint32_t sf = tmem + TMEM_SF;
+        for (int j = 0; j < kAtomsPerStage<MX>; ++j) {  // the MMAs below follow these copies in issue order
+            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
+            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
+            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
+        }
+        const uint64_t t0 = clock64();
+        for (int64_t it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t acc = (it > 0 || j > 0) ? 1u : 0u;
+                if (MX)
+                    tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * (j >> 1), sf + 16 + 8 * (j >> 1), acc,
+                                  idesc_mx(2u * (uint32_t)(j & 1)));
+                else
+                    tc_mma_if<MX>(issue, tmem, da + 2 * j, db + 2 * j, sf + 4 * j, sf + 16 + 8 * j, acc, IDESC);
+            }
+            tc_commit_self_if(issue, bar_round);
+            __syncwarp();
+        }
+        tc_commit_self_if(issue, bar_drain);
+        const bool ok = mbar_wait_warp(bar_drain, 0, abort_flag, false);
+        const uint64_t t1 = clock64();
+        if (lane == 0) {
+            cycles[cluster_id_x()] = t1 - t0;
+            if (!ok) atomicExch(status, kTimeoutStatus);
+        }
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+}
+
+template <bool MX>
+cudaError_t launch_mma_rate_t(int64_t iters, uint64_t *cycles, int64_t cycles_len, int *pairs_out, int *status,
+                              cudaStream_t s, int *launches) {
+    cudaError_t e = cudaFuncSetAttribute(mma_rate_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, PROBE_SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
+    cfg.blockDim = dim3(PROBE_THREADS);
+    cfg.dynamicSmemBytes = PROBE_SMEM;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mma_rate_kernel<MX>, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms() / 2;
+    }
+    if (n > cycles_len) return cudaErrorInvalidValue;
+    *pairs_out = n;
+    mma_rate_kernel<MX><<<2 * n, PROBE_THREADS, PROBE_SMEM, s>>>(cycles, iters, status);
+    ++*launches;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
@@ -937,6 +1044,12 @@ cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s, int *launches) {
         return cudaMemset2DAsync(a.C, (size_t)a.ldc * esz, 0, (size_t)a.N * esz, (size_t)a.M, s);
     }
     return a.mx ? launch_gemm_t<true>(a, s, launches) : launch_gemm_t<false>(a, s, launches);
+}
+
+cudaError_t launch_mma_rate(bool mx, int64_t iters, uint64_t *cycles, int64_t cycles_len, int *pairs_out, int *status,
+                            cudaStream_t s, int *launches) {
+    return mx ? launch_mma_rate_t<true>(iters, cycles, cycles_len, pairs_out, status, s, launches)
+              : launch_mma_rate_t<false>(iters, cycles, cycles_len, pairs_out, status, s, launches);
 }
 
 }  // namespace nvfp4

@@ -88,6 +88,9 @@ cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_ou
 
 // One bounded wait on an mbarrier nothing arrives on; records the timeout status.
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);
+// Tensor-pipe rate probe (gemm.cu): one launch over every co-resident CTA pair.
+cudaError_t launch_mma_rate(bool mx, int64_t iters, uint64_t *cycles, int64_t cycles_len, int *pairs_out, int *status,
+                            cudaStream_t s, int *launches);
 
 // relu^2 (dh == nullptr) or its derivative over a contiguous [R x C] bf16 tensor (R % 16 == 0,
 // C % 8 == 0), also writing max |out| and max |RHT(out)| (transform down 16-row groups);

@@ -159,6 +159,22 @@ def test_selftest_rejections(lib):
     assert lib.nvfp4_selftest_wait_timeout(ws, 256, 3_000_000_000, None) == binding.NVFP4_ERR_INVALID_ARG
 
 
+def test_mma_rate_probe_rejections(lib):
+    ws, cyc, pairs = C.c_void_p(0x20000), C.c_void_p(0x40000), C.c_int(0)
+    f = lib.nvfp4_selftest_mma_rate
+    f.argtypes = [C.c_int, C.c_int64, C.c_void_p, C.c_int64, C.POINTER(C.c_int), C.c_void_p, C.c_size_t, C.c_void_p]
+    E = binding
+    assert f(0, 10, None, 74, C.byref(pairs), ws, 256, None) == E.NVFP4_ERR_INVALID_ARG      # no output buffer
+    assert f(0, 10, cyc, 74, None, ws, 256, None) == E.NVFP4_ERR_INVALID_ARG                 # no pair count
+    assert f(2, 10, cyc, 74, C.byref(pairs), ws, 256, None) == E.NVFP4_ERR_INVALID_ARG       # mx not 0/1
+    assert f(0, 0, cyc, 74, C.byref(pairs), ws, 256, None) == E.NVFP4_ERR_INVALID_ARG        # iters < 1
+    assert f(1, 1000001, cyc, 74, C.byref(pairs), ws, 256, None) == E.NVFP4_ERR_INVALID_ARG  # iters too many
+    assert f(0, 10, cyc, 74, C.byref(pairs), None, 256, None) == E.NVFP4_ERR_WORKSPACE
+    assert f(0, 10, cyc, 74, C.byref(pairs), ws, 255, None) == E.NVFP4_ERR_WORKSPACE
+    assert f(0, 10, cyc, 74, C.byref(pairs), C.c_void_p(0x20008), 256, None) == E.NVFP4_ERR_ALIGNMENT
+    assert f(0, 10, C.c_void_p(0x40004), 74, C.byref(pairs), ws, 256, None) == E.NVFP4_ERR_ALIGNMENT
+
+
 def test_quantize_dual_rejections(lib):
     ws = C.c_void_p(0x20000)
     row, col = _tensor(64, 64), _tensor(64, 64)
