@@ -39,6 +39,7 @@ M_TOK, HID, FFN = W.TOKENS, W.HIDDEN, W.FFN
 GEMM_FLOPS = 6 * 2 * M_TOK * HID * FFN            # 1.031e13 per step per GPU
 SEED = 1234
 MMA_ROUND_FLOP = 4 * 2 * 256 * 256 * 64          # one probe round of a CTA pair
+HBM_NOMINAL_GBS = 8000.0                          # B200 HBM3e, nominal
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 FP4_PER_BF16 = 4.0                                 # nominal dense ratio 9 / 2.25 PFLOP/s
 FP4_NOMINAL_TFLOPS = 9000.0                        # B200 dense FP4, vendor figure
@@ -509,6 +510,7 @@ def run_ours(args):
                                   "bytes_per_elem": {"single": QUANT_BYTES_SINGLE, "dual": QUANT_BYTES_DUAL,
                                                      "amax_supplied": QUANT_BYTES_AMAX_IN},
                                   "calls_per_step": q[2] // args.steps, "peak_source": src + " hbm_gbs",
+                                  "frac_of_nominal_8tbs": q_gbs / HBM_NOMINAL_GBS,
                                   "call_ms": q[0] / q[2]},
             "mxfp4_quantize": {"tensor": "h %dx%d bf16, rowwise" % tuple(hten.shape), "us_per_call": mx_us,
                                "achieved": hten.numel() * MX_BYTES / (mx_us * 1e-6) / 1e9, "unit": "GB/s",

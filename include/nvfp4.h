@@ -63,7 +63,8 @@ typedef enum nvfp4_status {
     NVFP4_ERR_WORKSPACE = 4,          /* workspace missing or smaller than required             */
     NVFP4_ERR_UNSUPPORTED_DEVICE = 5, /* current device is not compute capability 10.0          */
     NVFP4_ERR_CUDA = 6,               /* a CUDA runtime call or launch failed                   */
-    NVFP4_ERR_DEVICE_TIMEOUT = 7      /* a bounded device-side wait expired (see nvfp4_check)   */
+    NVFP4_ERR_DEVICE_TIMEOUT = 7,     /* a bounded device-side wait expired (see nvfp4_check)   */
+    NVFP4_ERR_DEVICE_BOUNDS = 8       /* checked build: a kernel index fell outside its buffer  */
 } nvfp4_status;
 
 typedef enum nvfp4_dtype {
@@ -376,6 +377,30 @@ NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(void *workspace, size_t ws_by
  * NVFP4_ERR_WORKSPACE, NVFP4_ERR_ALIGNMENT, NVFP4_ERR_UNSUPPORTED_DEVICE. */
 NVFP4_API nvfp4_status nvfp4_selftest_mma_rate(int mx, int64_t iters, uint64_t *cycles, int64_t cycles_len,
                                                int *pairs_out, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Bounds-checked debug build (libnvfp4_checked.so, compiled with
+ * -DNVFP4_BOUNDS_CHECK; no counterpart on the pages: it checks the library's
+ * own index arithmetic).  There every guarded global access of the kernels
+ * first checks the elements it touches against the extent of the buffer as the
+ * call's shapes define it; an access that would fall outside is skipped and
+ * the source line of the first such check is recorded (nothing traps).
+ * nvfp4_bounds_status synchronises the device, reads and clears these records:
+ * NVFP4_ERR_DEVICE_BOUNDS with *site = file * 100000 + line (file: 1
+ * quantize.cu, 2 elementwise.cu, 3 gemm.cu, 4 selftest.cu) if a check failed
+ * since the last call, else NVFP4_OK with *site = 0.  *checked (host memory)
+ * is 1 in the checked build, 0 in the product build, which records nothing.
+ * Errors: NVFP4_ERR_INVALID_ARG (null pointer), NVFP4_ERR_CUDA. */
+NVFP4_API nvfp4_status nvfp4_bounds_status(int *checked, int *site);
+
+/* Self-test of that record (checked build only): one thread makes a check of
+ * element 0 of [0, n), which passes and sets buf[0] = 1, and a check of element
+ * n, which fails, so buf[n] is not written and the next nvfp4_bounds_status
+ * reports it.  buf: device memory of n + 1 bytes (the byte past the checked
+ * range exists, so even an unguarded write would stay inside the allocation),
+ * caller-owned; 1 <= n.  Asynchronous.  Errors: NVFP4_ERR_INVALID_ARG (null
+ * buf, n < 1, or the product build, where it launches nothing),
+ * NVFP4_ERR_UNSUPPORTED_DEVICE, NVFP4_ERR_CUDA. */
+NVFP4_API nvfp4_status nvfp4_selftest_bounds(uint8_t *buf, int64_t n, cudaStream_t stream);
 
 /* Number of kernel launches the most recent successful call on this host
  * thread issued (launch accounting for benchmarks). */

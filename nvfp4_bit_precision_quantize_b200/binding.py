@@ -11,7 +11,9 @@ from dataclasses import dataclass
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
+# NVFP4_CHECKED=1 selects the bounds-checked debug build (build.build(checked=True)).
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libnvfp4_checked.so" if os.environ.get("NVFP4_CHECKED") == "1" else "libnvfp4.so")
 
 NVFP4_OK = 0
 NVFP4_ERR_INVALID_ARG = 1
@@ -21,6 +23,7 @@ NVFP4_ERR_WORKSPACE = 4
 NVFP4_ERR_UNSUPPORTED_DEVICE = 5
 NVFP4_ERR_CUDA = 6
 NVFP4_ERR_DEVICE_TIMEOUT = 7
+NVFP4_ERR_DEVICE_BOUNDS = 8
 
 NVFP4_DTYPE_F32 = 0
 NVFP4_DTYPE_BF16 = 1
@@ -37,7 +40,8 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_quantize_dual_workspace_size", "nvfp4_quantize_dual", "nvfp4_relu2_fwd_amax",
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
            "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
-           "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd", "nvfp4_selftest_mma_rate")
+           "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd", "nvfp4_selftest_mma_rate",
+           "nvfp4_bounds_status", "nvfp4_selftest_bounds")
 
 
 class CTensor(C.Structure):
@@ -85,6 +89,8 @@ def load():
         "nvfp4_linear_fwd_noalloc": (i32, [vp, vp, vp, i64, i64, i64, i32, i32, vp]),
         "nvfp4_selftest_wait_timeout": (i32, [vp, sz, u64, vp]),
         "nvfp4_selftest_mma_rate": (i32, [i32, i64, vp, i64, C.POINTER(C.c_int), vp, sz, vp]),
+        "nvfp4_bounds_status": (i32, [C.POINTER(C.c_int), C.POINTER(C.c_int)]),
+        "nvfp4_selftest_bounds": (i32, [vp, i64, vp]),
         "nvfp4_quantize_dual_workspace_size": (sz, []),
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
         "nvfp4_relu2_fwd_amax": (i32, [vp, vp, i64, vp, vp, sz, vp]),
@@ -543,6 +549,25 @@ def nvfp4_selftest_mma_rate(cycles, ws, iters, mx=False, stream=None):
     _ok(load().nvfp4_selftest_mma_rate(1 if mx else 0, int(iters), _ptr(cycles), cycles.numel(), C.byref(pairs),
                                        _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_selftest_mma_rate")
     return pairs.value
+
+
+def nvfp4_bounds_status():
+    """(checked_build, site, status) from the bounds-checked build's records (read and
+    cleared); in the product build (False, 0, NVFP4_OK)."""
+    checked, site = C.c_int(0), C.c_int(0)
+    st = load().nvfp4_bounds_status(C.byref(checked), C.byref(site))
+    if st not in (NVFP4_OK, NVFP4_ERR_DEVICE_BOUNDS):
+        raise NVFP4Error(st, "nvfp4_bounds_status")
+    return bool(checked.value), site.value, st
+
+
+def nvfp4_selftest_bounds(buf, stream=None):
+    """Checked build only: one passing and one failing index check on a uint8 device
+    tensor of n + 1 bytes (n = buf.numel() - 1)."""
+    _on_device(buf)
+    if buf.dtype != torch.uint8 or buf.numel() < 2:
+        raise ValueError("buf must be a uint8 tensor of at least 2 bytes")
+    _ok(load().nvfp4_selftest_bounds(_ptr(buf), buf.numel() - 1, _stream(stream)), "nvfp4_selftest_bounds")
 
 
 def nvfp4_last_launch_count():

@@ -615,6 +615,36 @@ nvfp4_status nvfp4_selftest_mma_rate(int mx, int64_t iters, uint64_t *cycles, in
                                                static_cast<int *>(workspace), stream, &call.launches)));
 }
 
+#ifdef NVFP4_BOUNDS_CHECK
+constexpr int kCheckedBuild = 1;
+#else
+constexpr int kCheckedBuild = 0;
+#endif
+
+nvfp4_status nvfp4_bounds_status(int *checked, int *site) {
+    if (!checked || !site) return NVFP4_ERR_INVALID_ARG;
+    *checked = kCheckedBuild;
+    *site = 0;
+    if (!kCheckedBuild) return NVFP4_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
+    cudaError_t (*readers[4])(int *) = {read_bounds_quantize, read_bounds_elementwise, read_bounds_gemm,
+                                        read_bounds_selftest};
+    for (int f = 0; f < 4; ++f) {  // read (and clear) every record; report the first file's
+        int line = 0;
+        if (readers[f](&line) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (line && !*site) *site = (f + 1) * 100000 + line;
+    }
+    return *site ? NVFP4_ERR_DEVICE_BOUNDS : NVFP4_OK;
+}
+
+nvfp4_status nvfp4_selftest_bounds(uint8_t *buf, int64_t n, cudaStream_t stream) {
+    Call call(__func__);
+    if (!kCheckedBuild || !buf || n < 1) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    return call.done(from_cuda(launch_selftest_bounds(buf, n, stream, &call.launches)));
+}
+
 int nvfp4_last_launch_count(void) { return g_last_launches; }
 
 const char *nvfp4_status_string(nvfp4_status status) {
@@ -627,6 +657,7 @@ const char *nvfp4_status_string(nvfp4_status status) {
         case NVFP4_ERR_UNSUPPORTED_DEVICE: return "current device is not compute capability 10.0 (B200)";
         case NVFP4_ERR_CUDA: return "CUDA runtime error";
         case NVFP4_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+        case NVFP4_ERR_DEVICE_BOUNDS: return "a kernel index fell outside its buffer (bounds-checked build)";
     }
     return "unknown status";
 }

@@ -5,6 +5,7 @@
 // variants also return max |output| (of the stored bf16 values), one partial
 // per CTA reduced by a second one-CTA kernel, so that the NVFP4 quantisation
 // that follows can skip its own amax pass (tensor scale from a supplied amax).
+#include "checked.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,7 +25,7 @@ __device__ __forceinline__ void write_partial(float m, float *partials) {
     if (threadIdx.x == 0) {
         float b = 0.0f;
         for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
-        partials[blockIdx.x] = b;
+        if (NVFP4_IN_RANGE(blockIdx.x, 1, kMaxPartials)) partials[blockIdx.x] = b;
     }
 }
 
@@ -34,12 +35,14 @@ __global__ void __launch_bounds__(kThreads) relu2_fwd_kernel(const uint16_t *__r
     const int64_t nv = n / 8, stride = (int64_t)gridDim.x * kThreads;
     float m = 0.0f;
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nv; i += stride) {
+        if (!NVFP4_IN_RANGE(8 * i, 8, n)) continue;
         const uint4 v = ldg_stream(y + 8 * i);
         const uint4 o = make_uint4(relu2_pair(v.x), relu2_pair(v.y), relu2_pair(v.z), relu2_pair(v.w));
         reinterpret_cast<uint4 *>(h)[i] = o;
         if (AMAX) m = absmax_pair(absmax_pair(absmax_pair(absmax_pair(m, o.x), o.y), o.z), o.w);
     }
     for (int64_t i = 8 * nv + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
+        if (!NVFP4_IN_RANGE(i, 1, n)) continue;
         const float a = relu(__uint_as_float((uint32_t)y[i] << 16));
         const uint16_t o = bf16_of(__fmul_rn(a, a));
         h[i] = o;
@@ -55,6 +58,7 @@ __global__ void __launch_bounds__(kThreads) relu2_bwd_kernel(const uint16_t *__r
     const int64_t nv = n / 8, stride = (int64_t)gridDim.x * kThreads;
     float m = 0.0f;
     for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nv; i += stride) {
+        if (!NVFP4_IN_RANGE(8 * i, 8, n)) continue;
         const uint4 g = ldg_stream(dh + 8 * i), v = ldg_stream(y + 8 * i);
         const uint4 o =
             make_uint4(drelu2_pair(g.x, v.x), drelu2_pair(g.y, v.y), drelu2_pair(g.z, v.z), drelu2_pair(g.w, v.w));
@@ -62,6 +66,7 @@ __global__ void __launch_bounds__(kThreads) relu2_bwd_kernel(const uint16_t *__r
         if (AMAX) m = absmax_pair(absmax_pair(absmax_pair(absmax_pair(m, o.x), o.y), o.z), o.w);
     }
     for (int64_t i = 8 * nv + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
+        if (!NVFP4_IN_RANGE(i, 1, n)) continue;
         const float g = __fmul_rn(2.0f, relu(__uint_as_float((uint32_t)y[i] << 16)));
         const uint16_t o = bf16_of(__fmul_rn(__uint_as_float((uint32_t)dh[i] << 16), g));
         dy[i] = o;
@@ -98,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 2) relu2_amax_rht_kernel(const uint1
     for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total; u += (int64_t)gridDim.x * kThreads) {
         const int64_t g = u / chunks, cc = u - g * chunks;
         const int64_t base = g * 16 * C + cc * 4;
+        if (!NVFP4_IN_RANGE(base, 15 * C + 4, R * C)) continue;  // the unit's 16 rows x 4 columns
         uint2 o[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -213,5 +219,7 @@ cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_ou
     ++*launches;
     return cudaGetLastError();
 }
+
+NVFP4_DEFINE_BOUNDS_READER(read_bounds_elementwise)
 
 }  // namespace nvfp4

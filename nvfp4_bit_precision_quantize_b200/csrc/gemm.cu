@@ -57,6 +57,7 @@
 
 #include <algorithm>
 
+#include "checked.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -792,8 +793,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 a = fmaxf(a, red[i]);
                 b = fmaxf(b, red[EPI_WARPS + i]);
             }
-            p.partials[blockIdx.x] = a;
-            p.partials[kMaxPartials + blockIdx.x] = __fmul_rn(b, 0.25f);  // max |z / 4| = RN(max |z| / 4)
+            if (NVFP4_IN_RANGE(blockIdx.x, 1, kMaxPartials)) {
+                p.partials[blockIdx.x] = a;
+                p.partials[kMaxPartials + blockIdx.x] = __fmul_rn(b, 0.25f);  // max |z / 4| = RN(max |z| / 4)
+            }
         }
     }
 
@@ -1051,5 +1054,7 @@ cudaError_t launch_mma_rate(bool mx, int64_t iters, uint64_t *cycles, int64_t cy
     return mx ? launch_mma_rate_t<true>(iters, cycles, cycles_len, pairs_out, status, s, launches)
               : launch_mma_rate_t<false>(iters, cycles, cycles_len, pairs_out, status, s, launches);
 }
+
+NVFP4_DEFINE_BOUNDS_READER(read_bounds_gemm)
 
 }  // namespace nvfp4

@@ -88,6 +88,12 @@ cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_ou
 
 // One bounded wait on an mbarrier nothing arrives on; records the timeout status.
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches);
+// Bounds-checked build: read and clear each translation unit's record (checked.cuh).
+cudaError_t read_bounds_quantize(int *site);
+cudaError_t read_bounds_elementwise(int *site);
+cudaError_t read_bounds_gemm(int *site);
+cudaError_t read_bounds_selftest(int *site);
+cudaError_t launch_selftest_bounds(uint8_t *buf, int64_t n, cudaStream_t s, int *launches);
 // Tensor-pipe rate probe (gemm.cu): one launch over every co-resident CTA pair.
 cudaError_t launch_mma_rate(bool mx, int64_t iters, uint64_t *cycles, int64_t cycles_len, int *pairs_out, int *status,
                             cudaStream_t s, int *launches);

@@ -15,6 +15,7 @@
 // operands: same page, section "Technologie stabilizujace proces treningowy".
 #include <algorithm>
 
+#include "checked.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,6 +23,15 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kThreads = 256;
+
+// Buffer extents for the bounds-checked build (arguments of NVFP4_IN_RANGE only).
+__host__ __device__ constexpr int64_t x_extent(int64_t R, int64_t C, int64_t ld) { return (R - 1) * ld + C; }
+__host__ __device__ constexpr int64_t nv_scales_extent(int64_t rows, int64_t k) {
+    return ((rows + 127) / 128) * 128 * (((k + 63) / 64) * 4);
+}
+__host__ __device__ constexpr int64_t mx_scales_extent(int64_t rows, int64_t k) {
+    return ((rows + 127) / 128) * 128 * (((k + 127) / 128) * 4);
+}
 
 // xor of a 16-byte row chunk with the sign-bit mask of Hadamard input row i
 // (bit i of the sign word set: every element of the chunk changes sign).
@@ -51,7 +61,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T *__restrict__ x,
         for (; i + (U - 1) * stride < total; i += U * stride) {
             uint4 raw[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) raw[u] = ldg_stream(x + (i + u * stride) * N);
+            for (int u = 0; u < U; ++u)
+                raw[u] = NVFP4_IN_RANGE((i + u * stride) * N, N, R * C) ? ldg_stream(x + (i + u * stride) * N) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 float v[N];
@@ -62,7 +73,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T *__restrict__ x,
         }
         for (; i < total; i += stride) {
             float v[N];
-            Vec<T>::unpack(ldg_stream(x + i * N), v);
+            Vec<T>::unpack(NVFP4_IN_RANGE(i * N, N, R * C) ? ldg_stream(x + i * N) : make_uint4(0u, 0u, 0u, 0u), v);
 #pragma unroll
             for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
         }
@@ -70,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T *__restrict__ x,
         for (; i < total; i += stride) {
             const int64_t r = i / chunks_per_row, c = (i - r * chunks_per_row) * N;
             float v[N];
-            Vec<T>::unpack(ldg_stream(x + r * ld + c), v);
+            Vec<T>::unpack(NVFP4_IN_RANGE(r * ld + c, N, x_extent(R, C, ld)) ? ldg_stream(x + r * ld + c) : make_uint4(0u, 0u, 0u, 0u), v);
 #pragma unroll
             for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
         }
@@ -82,7 +93,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T *__restrict__ x,
     if (threadIdx.x == 0) {
         float b = 0.0f;
         for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
-        partials[blockIdx.x] = b;
+        if (NVFP4_IN_RANGE(blockIdx.x, 1, kMaxPartials)) partials[blockIdx.x] = b;
     }
 }
 
@@ -107,7 +118,8 @@ __global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict_
         const T *p = x + (g * 16) * ld + cc * N;
         uint4 raw[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
+        for (int i = 0; i < 16; ++i)
+            raw[i] = NVFP4_IN_RANGE((g * 16 + i) * ld + cc * N, N, x_extent(R, C, ld)) ? ldg_stream(p + i * ld) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int i = 0; i < 16; ++i) raw[i] = xor4(raw[i], sign_mask<T>(signs, i));
 #pragma unroll
@@ -132,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) amax_rht_kernel(const T *__restrict_
     if (threadIdx.x == 0) {
         float b = 0.0f;
         for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, s_red[w]);
-        partials[blockIdx.x] = b;
+        if (NVFP4_IN_RANGE(blockIdx.x, 1, kMaxPartials)) partials[blockIdx.x] = b;
     }
 }
 
@@ -157,7 +169,8 @@ __global__ void __launch_bounds__(kThreads) amax_dual_kernel(const T *__restrict
         const T *p = x + (g * 16) * ld + cc * N;
         uint4 raw[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) raw[i] = ldg_stream(p + i * ld);
+        for (int i = 0; i < 16; ++i)
+            raw[i] = NVFP4_IN_RANGE((g * 16 + i) * ld + cc * N, N, x_extent(R, C, ld)) ? ldg_stream(p + i * ld) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int i = 0; i < 16; ++i) raw[i] = xor4(raw[i], sign_mask<T>(signs, i));
 #pragma unroll
@@ -192,8 +205,10 @@ __global__ void __launch_bounds__(kThreads) amax_dual_kernel(const T *__restrict
             b0 = fmaxf(b0, s_red[0][w]);
             b1 = fmaxf(b1, s_red[1][w]);
         }
-        partials_plain[blockIdx.x] = b0;
-        partials_rht[blockIdx.x] = b1;
+        if (NVFP4_IN_RANGE(blockIdx.x, 1, kMaxPartials)) {
+            partials_plain[blockIdx.x] = b0;
+            partials_rht[blockIdx.x] = b1;
+        }
     }
 }
 
@@ -345,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int64_t r = r0 + i;
-            if (b < KB && r < p.R) {
+            if (b < KB && r < p.R && NVFP4_IN_RANGE(r * p.ld + b * 16, 16, x_extent(p.R, p.C, p.ld))) {
                 load_block<LW>(xb + (r * p.ld + b * 16) * (int64_t)sizeof(T), a32, buf[i]);
             } else {
 #pragma unroll
@@ -384,11 +399,14 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
             uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
             if (SR) sr_words16((uint64_t)r * (uint64_t)K + (uint64_t)b * 16u, keys, w0, w1);
             const uint2 c = encode16<SR>(v, inv, w0, w1);
-            if (col_ok && r < p.R) *reinterpret_cast<uint2 *>(p.codes + r * (K / 2) + b * 8) = c;
+            if (col_ok && r < p.R && NVFP4_IN_RANGE(r * (K / 2) + b * 8, 8, p.R * (K / 2)))
+                *reinterpret_cast<uint2 *>(p.codes + r * (K / 2) + b * 8) = c;
             uint32_t word = sb << (8 * (lane & 3));
             word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
             word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-            if ((lane & 3) == 0 && atom < KB4)
+            if ((lane & 3) == 0 && atom < KB4 &&
+                NVFP4_IN_RANGE(((r >> 7) * KB4 + atom) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4, 4,
+                               nv_scales_extent(p.R, K)))
                 *reinterpret_cast<uint32_t *>(p.scales + ((r >> 7) * KB4 + atom) * 512 + (r & 31) * 16 +
                                               ((r >> 5) & 3) * 4) = word;
         }
@@ -452,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int64_t r = r_warp + i;
-        raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+        raw[i] = (col_ok && r < p.R && NVFP4_IN_RANGE(r * p.ld + c, N, x_extent(p.R, p.C, p.ld))) ? ldg_stream(x + r * p.ld + c)
+                                                                               : make_uint4(0u, 0u, 0u, 0u);
     }
     const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));
     float s_t_row = 0.0f;
@@ -485,7 +504,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int64_t r = rg + i;
-                raw[i] = (col_ok && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+                raw[i] = (col_ok && r < p.R && NVFP4_IN_RANGE(r * p.ld + c, N, x_extent(p.R, p.C, p.ld))) ? ldg_stream(x + r * p.ld + c)
+                                                                               : make_uint4(0u, 0u, 0u, 0u);
             }
         }
         if (DUAL) {
@@ -506,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
                 float q[N];
 #pragma unroll
                 for (int j = 0; j < N; ++j) q[j] = __fmul_rn(v[j], inv);
-                if (col_ok && r < p.R) {
+                if (col_ok && r < p.R && NVFP4_IN_RANGE(r * (p.C / 2) + c / 2, N / 2, p.R * (p.C / 2))) {
                     uint8_t *dst = p.row_codes + r * (p.C / 2) + c / 2;
                     if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q) & (inv == 0.0f ? 0x77777777u : ~0u);
                     else *reinterpret_cast<uint16_t *>(dst) =
@@ -579,7 +599,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
         const int l = cl / N, j = cl % N, q = j * P + pu;
         const int64_t orow = c0 + cl;
         const int64_t rem = p.R - (r0 + 32 * pu);
-        if (orow < p.C && rem > 0) {
+        if (orow < p.C && rem > 0 &&
+            NVFP4_IN_RANGE(orow * (K / 2) + (r0 / 2) + 16 * pu, rem >= 32 ? 16 : 8, p.C * (K / 2))) {
             const uint4 u = s_units[q * 32 + (l ^ (q & 7))];
             uint8_t *dst = p.codes + orow * (K / 2) + (r0 / 2) + 16 * pu;
             if (rem >= 32 && vec16) {
@@ -595,7 +616,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
         for (int i = threadIdx.x; i < ARR * ACR * 32; i += kThreads) {
             const int atom = i >> 5, ar = atom / ACR, ac = atom % ACR;
             const int64_t grow = by * ARR + ar, gcol = bx * ACR + ac;
-            if (grow < rowtiles_r && gcol < kb4_r) {
+            if (grow < rowtiles_r && gcol < kb4_r &&
+                NVFP4_IN_RANGE((grow * kb4_r + gcol) * 512 + (i & 31) * 16, 16, nv_scales_extent(p.R, p.C))) {
                 uint8_t *dst = p.row_scales + (grow * kb4_r + gcol) * 512 + (i & 31) * 16;
                 *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_scr + i * 16);
             }
@@ -606,7 +628,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
     for (int i = threadIdx.x; i < AR * AC * 32; i += kThreads) {
         const int atom = i >> 5, ar = atom / AC, ac = atom % AC;
         const int64_t grow = bx * AR + ar, gcol = by * AC + ac;
-        if (grow < rowtiles && gcol < KB4) {
+        if (grow < rowtiles && gcol < KB4 &&
+            NVFP4_IN_RANGE((grow * KB4 + gcol) * 512 + (i & 31) * 16, 16, nv_scales_extent(p.C, p.R))) {
             uint8_t *dst = p.scales + (grow * KB4 + gcol) * 512 + (i & 31) * 16;
             *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s_sc + i * 16);
         }
@@ -659,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const 
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int64_t r = r0 + i;
-            buf[i] = (c < p.C && r < p.R) ? ldg_stream(x + r * p.ld + c) : make_uint4(0u, 0u, 0u, 0u);
+            buf[i] = (c < p.C && r < p.R && NVFP4_IN_RANGE(r * p.ld + c, N, x_extent(p.R, p.C, p.ld))) ? ldg_stream(x + r * p.ld + c)
+                                                                                        : make_uint4(0u, 0u, 0u, 0u);
         }
     };
 
@@ -689,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const 
             float q[N];
 #pragma unroll
             for (int j = 0; j < N; ++j) q[j] = __fmul_rn(v[j], inv);
-            if (col_ok && r < p.R) {
+            if (col_ok && r < p.R && NVFP4_IN_RANGE(r * (K / 2) + c / 2, N / 2, p.R * (K / 2))) {
                 uint8_t *dst = p.codes + r * (K / 2) + c / 2;
                 if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
                 else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
@@ -703,7 +727,9 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const 
         const int64_t atom0 = tc * ATOMS;
         for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
             const int atom = i >> 5;
-            if (atom0 + atom < KB4) {
+            if (atom0 + atom < KB4 &&
+                NVFP4_IN_RANGE(((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half, 8,
+                               mx_scales_extent(p.R, p.C))) {
                 const int off = atom * 512 + (i & 31) * 16 + 8 * half;
                 uint8_t *dst = p.scales + ((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half;
                 *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(s_sc + off);
@@ -739,7 +765,7 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_mx_kernel(const MxP
     uint2 raw[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-        raw[i] = (rows_ok && c0 < p.C) ? __ldg(reinterpret_cast<const uint2 *>(x + (r0 + i) * p.ld + c0))
+        raw[i] = (rows_ok && c0 < p.C && NVFP4_IN_RANGE((r0 + i) * p.ld + c0, CPT, x_extent(p.R, p.C, p.ld))) ? __ldg(reinterpret_cast<const uint2 *>(x + (r0 + i) * p.ld + c0))
                                        : make_uint2(0u, 0u);
     const int64_t b = r0 / 32;                 // 32-block index along k
 #pragma unroll
@@ -762,11 +788,13 @@ __global__ void __launch_bounds__(kThreads) quantize_colwise_mx_kernel(const MxP
         const float inv = __uint_as_float((254u - code) << 23);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
-        if (rows_ok && c < p.C) {
+        if (rows_ok && c < p.C && NVFP4_IN_RANGE(c * (K / 2) + r0 / 2, 16, p.C * (K / 2))) {
             const uint4 u = make_uint4(e2m1x8(v), e2m1x8(v + 8), e2m1x8(v + 16), e2m1x8(v + 24));
             *reinterpret_cast<uint4 *>(p.codes + c * (K / 2) + r0 / 2) = u;
         }
-        p.scales[((c >> 7) * KB4 + (b >> 2)) * 512 + (c & 31) * 16 + ((c >> 5) & 3) * 4 + (b & 3)] = (uint8_t)code;
+        if (NVFP4_IN_RANGE(((c >> 7) * KB4 + (b >> 2)) * 512 + (c & 31) * 16 + ((c >> 5) & 3) * 4 + (b & 3), 1,
+                           mx_scales_extent(p.C, K)))
+            p.scales[((c >> 7) * KB4 + (b >> 2)) * 512 + (c & 31) * 16 + ((c >> 5) & 3) * 4 + (b & 3)] = (uint8_t)code;
     }
 }
 
@@ -894,5 +922,7 @@ cudaError_t launch_quantize(const QuantizeArgs &a, cudaStream_t s, int *launches
     }
     return a.bf16 ? run<uint16_t>(a, s, launches) : run<float>(a, s, launches);
 }
+
+NVFP4_DEFINE_BOUNDS_READER(read_bounds_quantize)
 
 }  // namespace nvfp4

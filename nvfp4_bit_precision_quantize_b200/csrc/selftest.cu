@@ -6,6 +6,7 @@
 // NVFP4_ERR_DEVICE_TIMEOUT in the workspace status word and returns, leaving
 // the context usable.  The pages have no counterpart: this checks the
 // library's own error plumbing.
+#include "checked.cuh"
 #include "internal.h"
 
 namespace nvfp4 {
@@ -33,7 +34,22 @@ __global__ void wait_timeout_kernel(int *status, uint64_t limit_ns) {
     atomicExch(status, 7);  // NVFP4_ERR_DEVICE_TIMEOUT
 }
 
+// One check that passes (element 0) and one that fails (element n of an
+// n-element range); buf holds n + 1 bytes.
+__global__ void bounds_selftest_kernel(uint8_t *buf, int64_t n) {
+    if (NVFP4_IN_RANGE(0, 1, n)) buf[0] = 1;
+    if (NVFP4_IN_RANGE(n, 1, n)) buf[n] = 1;
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_bounds(uint8_t *buf, int64_t n, cudaStream_t s, int *launches) {
+    bounds_selftest_kernel<<<1, 1, 0, s>>>(buf, n);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+NVFP4_DEFINE_BOUNDS_READER(read_bounds_selftest)
 
 cudaError_t launch_wait_timeout(int *status, uint64_t limit_ns, cudaStream_t s, int *launches) {
     wait_timeout_kernel<<<1, 1, 0, s>>>(status, limit_ns);

@@ -37,6 +37,30 @@ def test_exports_every_declared_function(lib):
     assert set(names) == set(binding.EXPORTS)
 
 
+def test_checked_build_exports_and_reports(lib):
+    """The bounds-checked debug build exports the same functions; the product build
+    records nothing and refuses the bounds self-test."""
+    path = build.build(checked=True)
+    L = C.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    checked, site = C.c_int(-1), C.c_int(-1)
+    f = lib.nvfp4_bounds_status
+    f.argtypes = [C.POINTER(C.c_int), C.POINTER(C.c_int)]
+    assert f(C.byref(checked), C.byref(site)) == binding.NVFP4_OK and (checked.value, site.value) == (0, 0)
+    assert f(None, C.byref(site)) == binding.NVFP4_ERR_INVALID_ARG
+    lib.nvfp4_selftest_bounds.argtypes = [C.c_void_p, C.c_int64, C.c_void_p]
+    assert lib.nvfp4_selftest_bounds(C.c_void_p(0x20000), 16, None) == binding.NVFP4_ERR_INVALID_ARG
+    g = L.nvfp4_bounds_status
+    g.argtypes = [C.POINTER(C.c_int), C.POINTER(C.c_int)]
+    st = g(C.byref(checked), C.byref(site))
+    assert checked.value == 1
+    assert st in (binding.NVFP4_OK, binding.NVFP4_ERR_CUDA)  # NVFP4_ERR_CUDA where no GPU is present
+    L.nvfp4_selftest_bounds.argtypes = [C.c_void_p, C.c_int64, C.c_void_p]
+    assert L.nvfp4_selftest_bounds(None, 16, None) == binding.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_selftest_bounds(C.c_void_p(0x20000), 0, None) == binding.NVFP4_ERR_INVALID_ARG
+
+
 def test_sizes(lib):
     assert lib.nvfp4_codes_bytes(256, 256) == 256 * 128
     for rows, k in [(1, 16), (128, 64), (129, 64), (200, 272), (8192, 5120), (0, 64), (64, 0)]:
