@@ -272,16 +272,8 @@ __device__ __forceinline__ uint64_t f2(float lo, float hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
     return d;
 }
-__device__ __forceinline__ float f2lo(uint64_t d) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
-    return lo;
-}
-__device__ __forceinline__ float f2hi(uint64_t d) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
-    return hi;
-}
+__device__ __forceinline__ float f2lo(uint64_t d) { return __uint_as_float((uint32_t)d); }
+__device__ __forceinline__ float f2hi(uint64_t d) { return __uint_as_float((uint32_t)(d >> 32)); }
 __device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));

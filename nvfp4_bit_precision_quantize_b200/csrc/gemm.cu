@@ -295,17 +295,6 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[3
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart (SBO); LBO unused; version 1 (sm_100).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
@@ -685,15 +674,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t row_sign = p.epi != GEMM_EPI_PLAIN ? ((rht_sign_bits(p.seed) >> (lane & 15)) & 1u) << 31 : 0u;
         int tile_i = 0;
         for (int t = cid; t < p.num_tiles; t += ncl, ++tile_i) {
-            bool ok = mbar_wait(bar_accf, tile_i & 1, abort_flag);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (!ok) break;
-            tc_fence_after();
+            // the tile's coordinates before the wait: off the accumulator hand-off path
             int mt, nt;
             tile_coords(p, t, mt, nt);
             const int row0 = mt * BM + 128 * (int)rank + (int)q * 32;  // this warp's 32 rows
             const int col0 = nt * BN + 128 * hh;                        // and 128 columns
             const bool rows_in = row0 < p.M;
+            bool ok = mbar_wait(bar_accf, tile_i & 1, abort_flag);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) break;
+            tc_fence_after();
             if (p.c_bf16) {
                 // All 128 accumulator columns into registers, TMEM handed back, then
                 // scaled and packed to bf16, each 64-column chunk out through the
@@ -755,20 +745,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                 }
             } else {
-                // f32: four 32-column chunks; TMEM handed back after the last read
+                // f32: four 32-column chunks, read two at a time; TMEM handed back once
+                // the second pair is in registers
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + 32 * c, r);
-                    if (c == 3) {
+                for (int c = 0; c < 4; c += 2) {
+                    uint32_t r[2][32];
+                    tmem_ld32_nowait(tbase + 32 * c, r[0]);
+                    tmem_ld32_nowait(tbase + 32 * (c + 1), r[1]);
+                    tmem_wait_ld();
+                    if (c == 2) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_remote(mapa(bar_acce, 0));
                     }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__fmul_rn(__uint_as_float(r[j]), scale));
-                    const int x = col0 + 32 * c;
-                    store_chunk(&map_c, stg, r, lane, x, row0, rows_in && x < p.N);
+                    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            r[u][j] = __float_as_uint(__fmul_rn(__uint_as_float(r[u][j]), scale));
+                        const int x = col0 + 32 * (c + u);
+                        store_chunk(&map_c, stg, r[u], lane, x, row0, rows_in && x < p.N);
+                    }
                 }
             }
         }
