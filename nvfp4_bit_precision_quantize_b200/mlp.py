@@ -149,3 +149,19 @@ class MlpStep:
         """Forward and backward; X, dY2 and the output Y2 default to the step's own buffers."""
         self.forward(X, Y2, ev=ev, bytes_per_elem=bytes_per_elem)
         self.backward(X, dY2, ev=ev, bytes_per_elem=bytes_per_elem, grad_ready=grad_ready)
+
+    def capture(self, stream=None):
+        """The step on its own buffers (inputs["X"], inputs["dY2"], self.Y2 ...) captured once in
+        a CUDA graph; returns the graph, whose replay() runs the same 24 kernels with the same
+        arguments.  A loop copies each step's inputs into those buffers and replays.  The
+        step is run once eagerly first (the library's per-device set-up happens outside the
+        capture).  The gradient exchange is not captured: call it after replay()."""
+        s = stream if stream is not None else torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.step()
+        torch.cuda.current_stream().wait_stream(s)
+        return g
