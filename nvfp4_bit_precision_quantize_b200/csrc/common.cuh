@@ -151,18 +151,27 @@ __device__ __forceinline__ uint32_t e2m1x8(const float *v) {
 // the binary32 grid has x > t iff roundup(x) > t), and 1 is subtracted again
 // (exact).  Magnitudes are first clamped to 7: everything from 6 up lands on 6
 // or 8, which the saturating E2M1 conversion turns into 6.
-// `carry` = (2^16 - 1 - rnd16) * 2^6 + 63 (sr_carry_lo / sr_carry_hi below).
+// The constant is (2^16 - 1 - rnd16) * 2^6 + 63 = 2^22 - 1 - 64 rnd16, applied as
+// an integer multiply-add.  The "+1 below 1" offset is sat(2^24 - 2^24 a): for a
+// < 1 (a <= 1 - 2^-24) the exact value 2^24 (1 - a) is at least 1, for a >= 1 it
+// is at most 0, so one saturating FMA gives exactly 1 or 0.
 // Returns the E2M1 value (or 8 for 6), sign of r kept, for e2m1x*.
-__device__ __forceinline__ float sr_e2m1_value(float r, uint32_t carry) {
+__device__ __forceinline__ float sr_below_one(float a) {  // 1.0f if a < 1, else 0.0f (a finite, >= 0)
+    return __saturatef(__fmaf_rn(-a, 16777216.0f, 16777216.0f));
+}
+__device__ __forceinline__ uint32_t sr_round_bits(uint32_t t_bits, uint32_t rnd16) {
+    return (t_bits + 0x3FFFFFu + rnd16 * 0xFFFFFFC0u) & 0xFFC00000u;  // + (2^22 - 1 - 64 rnd16), mod 2^32
+}
+__device__ __forceinline__ float sr_e2m1_value(float r, uint32_t rnd16) {
     const float a = fminf(fabsf(r), 7.0f);
-    const float base = a < 1.0f ? 1.0f : 0.0f;
+    const float base = sr_below_one(a);
     const float t = __fadd_ru(a, base);
-    const float up = __uint_as_float((__float_as_uint(t) + carry) & 0xFFC00000u);
+    const float up = __uint_as_float(sr_round_bits(__float_as_uint(t), rnd16));
     return copysignf(__fsub_rn(up, base), r);
 }
-// carry of the low / high 16-bit draw of a Philox output word
-__device__ __forceinline__ uint32_t sr_carry_lo(uint32_t w) { return ((~w & 0xFFFFu) << 6) | 63u; }
-__device__ __forceinline__ uint32_t sr_carry_hi(uint32_t w) { return ((~w >> 16) << 6) | 63u; }
+// the low / high 16-bit draw of a Philox output word
+__device__ __forceinline__ uint32_t sr_rnd_lo(uint32_t w) { return w & 0xFFFFu; }
+__device__ __forceinline__ uint32_t sr_rnd_hi(uint32_t w) { return w >> 16; }
 
 // ---------------------------------------------------------------------------
 // Per-block scale:  sb = E4M3(RN(RN(amax_b / 6) / s_t)),  dec = e4m3(sb) * s_t,

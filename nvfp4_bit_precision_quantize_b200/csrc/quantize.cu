@@ -24,6 +24,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
+#ifdef NVFP4_BOUNDS_CHECK
 // Buffer extents for the bounds-checked build (arguments of NVFP4_IN_RANGE only).
 __host__ __device__ constexpr int64_t x_extent(int64_t R, int64_t C, int64_t ld) { return (R - 1) * ld + C; }
 __host__ __device__ constexpr int64_t nv_scales_extent(int64_t rows, int64_t k) {
@@ -32,6 +33,7 @@ __host__ __device__ constexpr int64_t nv_scales_extent(int64_t rows, int64_t k) 
 __host__ __device__ constexpr int64_t mx_scales_extent(int64_t rows, int64_t k) {
     return ((rows + 127) / 128) * 128 * (((k + 127) / 128) * 4);
 }
+#endif
 
 // xor of a 16-byte row chunk with the sign-bit mask of Hadamard input row i
 // (bit i of the sign word set: every element of the chunk changes sign).
@@ -244,9 +246,9 @@ __device__ __forceinline__ void sr_words16(uint64_t idx0, const PhiloxKeys &k, u
     w0 = philox4x32_10(make_uint4((uint32_t)c, (uint32_t)(c >> 32), 0u, 0u), k);
     w1 = philox4x32_10(make_uint4((uint32_t)(c + 1), (uint32_t)((c + 1) >> 32), 0u, 0u), k);
 }
-__device__ __forceinline__ uint32_t sr_carry(const uint4 &w, int e) {  // e = idx & 7, compile-time after unrolling
+__device__ __forceinline__ uint32_t sr_draw(const uint4 &w, int e) {  // e = idx & 7, compile-time after unrolling
     const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
-    return (e & 1) ? sr_carry_hi(word) : sr_carry_lo(word);
+    return (e & 1) ? sr_rnd_hi(word) : sr_rnd_lo(word);
 }
 
 // 16 E2M1 codes of one block (element 0 in the lowest nibble of .x), from the
@@ -265,11 +267,11 @@ __device__ __forceinline__ uint2 encode16_x2(const uint64_t (&p)[8], float inv, 
         const float r0 = f2lo(r), r1 = f2hi(r);
         if (SR) {
             const float a0 = fminf(fabsf(r0), 7.0f), a1 = fminf(fabsf(r1), 7.0f);
-            const uint64_t base = f2(a0 < 1.0f ? 1.0f : 0.0f, a1 < 1.0f ? 1.0f : 0.0f);
+            const uint64_t base = f2(sr_below_one(a0), sr_below_one(a1));
             const uint64_t t = add2_ru(f2(a0, a1), base);
-            const uint32_t c0 = sr_carry(k < 4 ? w0 : w1, (2 * k) & 7), c1 = sr_carry(k < 4 ? w0 : w1, (2 * k + 1) & 7);
-            const uint64_t up = f2(__uint_as_float((__float_as_uint(f2lo(t)) + c0) & 0xFFC00000u),
-                                   __uint_as_float((__float_as_uint(f2hi(t)) + c1) & 0xFFC00000u));
+            const uint32_t d0 = sr_draw(k < 4 ? w0 : w1, (2 * k) & 7), d1 = sr_draw(k < 4 ? w0 : w1, (2 * k + 1) & 7);
+            const uint64_t up = f2(__uint_as_float(sr_round_bits(__float_as_uint(f2lo(t)), d0)),
+                                   __uint_as_float(sr_round_bits(__float_as_uint(f2hi(t)), d1)));
             const uint64_t d = sub2_rn(up, base);
             q[2 * k] = copysignf(f2lo(d), r0);
             q[2 * k + 1] = copysignf(f2hi(d), r1);

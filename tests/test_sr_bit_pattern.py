@@ -22,19 +22,49 @@ import oracle
 GRID_CODE = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
 
 
+def below_one(a):
+    """The kernels' offset: sat(2^24 - 2^24 a) as one binary32 FMA (the exact value,
+    formed in float64 where it is exact for a binary32 a, rounded once)."""
+    v = (2.0 ** 24 - 2.0 ** 24 * np.asarray(a, dtype=np.float64)).astype(np.float32)
+    return np.clip(v, np.float32(0.0), np.float32(1.0)).astype(np.float32)
+
+
+def round_bits(t_bits, rnd16):
+    """The kernels' rounding step: bits + 2^22 - 1 - 64 rnd16 (mod 2^32), low 22 bits cleared."""
+    t_bits = np.asarray(t_bits, dtype=np.uint32)
+    rnd16 = np.asarray(rnd16, dtype=np.uint32)
+    with np.errstate(over="ignore"):
+        return (t_bits + np.uint32(0x3FFFFF) + rnd16 * np.uint32(0xFFFFFFC0)) & np.uint32(0xFFC00000)
+
+
+def test_offset_and_constant_forms():
+    """The offset equals [a < 1] for every binary32 a in [0, 8) on a dense sweep and at 1's
+    neighbours; the rounding constant equals the carry (2^16 - 1 - rnd16) * 2^6 + 63 for
+    every draw."""
+    a = np.arange(0, 0x41000000, 97, dtype=np.uint32).view(np.float32)
+    a = np.concatenate([a, np.float32([0.0, np.nextafter(np.float32(1), np.float32(0)), 1.0,
+                                       np.nextafter(np.float32(1), np.float32(2)), 7.0])])
+    assert np.array_equal(below_one(a), (a < np.float32(1.0)).astype(np.float32))
+    rnd = np.arange(65536, dtype=np.uint32)
+    carry = (((~rnd) & np.uint32(0xFFFF)) << np.uint32(6)) | np.uint32(63)
+    t = np.uint32(0x40E00000)  # 7.0
+    with np.errstate(over="ignore"):
+        assert np.array_equal(round_bits(np.full(rnd.shape, t), rnd), (t + carry) & np.uint32(0xFFC00000))
+    assert np.array_equal(np.uint32(0x3FFFFF) + rnd * np.uint32(0xFFFFFFC0), carry)
+
+
 def bit_pattern_sr(r, rnd16):
     """Codes from the kernels' bit-pattern SR decision (numpy restatement)."""
     r = np.asarray(r, dtype=np.float32)
     rnd16 = np.asarray(rnd16, dtype=np.uint32)
     a = np.minimum(np.abs(r), np.float32(7.0))
     small = a < np.float32(1.0)
-    base = np.where(small, np.float32(1.0), np.float32(0.0)).astype(np.float32)
+    base = below_one(a)
     # 1 + a rounded up to binary32 (exact in float64: a * 2^23 is an integer-valued double)
     up_sum = (1.0 + np.ceil(a.astype(np.float64) * 2.0 ** 23) / 2.0 ** 23).astype(np.float32)
     t = np.where(small, up_sum, a).astype(np.float32)
-    carry_in = (((~rnd16) & np.uint32(0xFFFF)) << np.uint32(6)) | np.uint32(63)
     with np.errstate(over="ignore"):
-        bits = (t.view(np.uint32) + carry_in) & np.uint32(0xFFC00000)
+        bits = round_bits(t.view(np.uint32), rnd16)
     mag = bits.view(np.float32) - base
     assert (mag <= np.float32(8.0)).all()
     mag = np.where(mag == np.float32(8.0), np.float32(6.0), mag)  # the conversion's saturation
