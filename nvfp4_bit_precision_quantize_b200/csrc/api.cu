@@ -189,6 +189,7 @@ nvfp4_status quantize_impl(const void *x, nvfp4_dtype dtype, int64_t R, int64_t 
     a.scales = out->scales;
     a.tensor_scale = out->tensor_scale;
     a.partials = ws ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kStatusBytes) : nullptr;
+    a.status = static_cast<int *>(ws);
     return from_cuda(launch_quantize(a, stream, launches));
 }
 

@@ -27,6 +27,7 @@ struct QuantizeArgs {
     uint8_t *scales;
     float *tensor_scale;
     float *partials;        // kMaxPartials floats (unused when amax_in is set)
+    int *status = nullptr;  // workspace status word (device timeouts), or null
 };
 
 // Rowwise RTN and colwise (RTN/SR, optional RHT) outputs of one tensor from one read.

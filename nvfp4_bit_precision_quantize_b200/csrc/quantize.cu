@@ -13,6 +13,9 @@
 // NVFP4 kontra ograniczenia mikroskalowania" (block 16, E4M3 block scale, FP32
 // tensor scale).  Hadamard transform and stochastic rounding on the Wgrad
 // operands: same page, section "Technologie stabilizujace proces treningowy".
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 
 #include "checked.cuh"
@@ -231,6 +234,7 @@ struct QParams {
     uint8_t *row_scales;
     float *row_tensor_scale;
     int aligned32;  // x and every row start 32-byte aligned (256-bit loads allowed)
+    int *status;    // workspace status word (device timeouts), or null
 };
 
 __device__ __forceinline__ float tensor_amax(const QParams &p, float *s_red) {
@@ -639,6 +643,221 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_colwise_kernel(const QPa
 }
 
 // ---------------------------------------------------------------------------
+// Pass 2, colwise, bf16 input fed by TMA.  Each warp works alone on tasks of
+// 64 input rows x 128 columns (four 16-row groups; lane l owns columns 4l ..
+// 4l+3): 128 output rows x 64 k, i.e. 32 code bytes per output row and exactly
+// one 512-byte scale atom.  Lane 0 keeps the next 16-row group in flight with a
+// 2-D TMA load (box 128 columns x 16 rows; rows and columns outside the tensor
+// arrive as zeros) into the warp's two-stage ring while the warp encodes the
+// current group from shared memory, so the loads never wait on the encode.
+// Each block is encoded exactly as in quantize_colwise_kernel (same steps, same
+// order).  Persistent: the CTA's set-up (tensor scale, element-scale tables,
+// Philox keys) happens once, and tasks run in reverse order (the tail of the
+// amax sweep is still in L2).  Every wait is bounded; on expiry the warp
+// records NVFP4_ERR_DEVICE_TIMEOUT, waits briefly for its loads in flight and
+// stops.
+// ---------------------------------------------------------------------------
+constexpr int kTmaWarps = 4;                        // warps per CTA
+constexpr int kTmaCols = 128;                       // columns per task
+constexpr int kTmaStageBytes = 16 * kTmaCols * 2;   // one 16-row group: 4 KB
+constexpr int kTmaStgBytes = 4 * 4 * 32 * 8;        // a task's codes, [group][column j][lane] x 8 bytes
+// Ring depth (groups in flight per warp) and CTAs per SM, measured per mode: round-to-nearest
+// is best with 16 warps per SM and two stages (h 8192x20480 with the RHT: 89 us against 93 with
+// three stages at 12 warps); stochastic rounding, bound by integer issue, with three stages at
+// 12 warps and up to 170 registers (dY 8192x20480: 191.5 us against 200.6).
+template <bool SR> __host__ __device__ constexpr int tma_stages() { return SR ? 3 : 2; }
+template <bool SR> __host__ __device__ constexpr int tma_ctas() { return SR ? 3 : 4; }
+template <bool SR> __host__ __device__ constexpr int tma_warp_bytes() {  // ring, codes, scale atom
+    return tma_stages<SR>() * kTmaStageBytes + kTmaStgBytes + 512;
+}
+template <bool SR> __host__ __device__ constexpr int tma_smem_bytes() {  // + alignment slack
+    return kTmaWarps * tma_warp_bytes<SR>() + 128;
+}
+constexpr uint64_t kTmaWaitNs = 2000000000ull, kTmaDrainNs = 20000000ull;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
+__device__ __forceinline__ bool q_mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __noinline__ bool q_mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (q_mbar_try(bar, parity)) return true;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > limit_ns) return false;
+    }
+}
+// Warp-uniform bounded wait: false on every lane if any lane gave up.
+__device__ __forceinline__ bool q_mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const bool ok = q_mbar_try(bar, parity) || q_mbar_wait_slow(bar, parity, limit_ns);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+// One 16-row group (box 128 x 16 bf16 = 4 KB) into a ring stage, completing on `bar`.
+__device__ __forceinline__ void q_tma_group(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kTmaStageBytes) : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"(map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+template <bool SR, bool RHT>
+__global__ void __launch_bounds__(32 * kTmaWarps, tma_ctas<SR>())
+    quantize_colwise_tma_kernel(const __grid_constant__ CUtensorMap map_x, const QParams p) {
+    constexpr int kTmaStages = tma_stages<SR>();
+    constexpr int kTmaWarpBytes = tma_warp_bytes<SR>();
+    extern __shared__ uint8_t q_smem_raw[];
+    uint8_t *q_smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q_smem_raw) + 127) & ~uintptr_t(127));
+    __shared__ float s_red[kTmaWarps];
+    __shared__ float s_inv[128], s_inv4[RHT ? 128 : 1];
+    __shared__ __align__(8) uint64_t s_bar[kTmaStages * kTmaWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *wsm = q_smem + warp * kTmaWarpBytes;
+    const uint32_t ring = smem_addr(wsm);
+    uint2 *stg = reinterpret_cast<uint2 *>(wsm + kTmaStages * kTmaStageBytes);
+    uint8_t *atom = wsm + kTmaStages * kTmaStageBytes + kTmaStgBytes;
+    const uint32_t bar = smem_addr(&s_bar[kTmaStages * warp]);
+    if (lane == 0) {
+        for (int i = 0; i < kTmaStages; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar + 8 * i) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const float s_t = tensor_scale_from_amax(tensor_amax(p, s_red));  // synchronises the CTA
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = s_t;
+    const ScaleCtx ctx = scale_ctx(s_t);
+    scale_table_init(s_inv, RHT ? s_inv4 : nullptr, s_t);
+    const uint32_t signs = RHT ? rht_sign_bits(p.seed) : 0u;
+    const bool fold = RHT && !SR && ctx.fast;  // quarter folded into the element scale (RTN only)
+    PhiloxKeys keys;
+    if (SR) keys = philox_keys(p.seed);
+    __syncthreads();
+
+    const int64_t K = p.R, KB4 = (K + 63) / 64;
+    const int64_t strips = (p.C + kTmaCols - 1) / kTmaCols, bands = (p.R + 63) / 64;
+    const int64_t ntasks = strips * bands;
+    const int64_t gw = (int64_t)blockIdx.x * kTmaWarps + warp, nw = (int64_t)gridDim.x * kTmaWarps;
+    const int64_t ngroups = gw < ntasks ? 4 * ((ntasks - 1 - gw) / nw + 1) : 0;
+    const bool vec16 = (K % 32) == 0;
+    // group q of this warp: task ntasks - 1 - gw - (q / 4) nw (band-major over strips), 16-row group q % 4
+    auto issue = [&](int64_t q) {
+        const int64_t t = ntasks - 1 - gw - (q >> 2) * nw;
+        const int64_t band = t / strips, strip = t - band * strips;
+        const uint32_t st = (uint32_t)(q % kTmaStages);
+        q_tma_group(ring + st * kTmaStageBytes, &map_x, bar + 8 * st, (int)(strip * kTmaCols),
+                    (int)(band * 64 + (q & 3) * 16));
+    };
+    if (lane == 0)
+        for (int64_t i = 0; i < kTmaStages && i < ngroups; ++i) issue(i);
+    int64_t q = 0;
+    for (; q < ngroups; ++q) {
+        const int64_t t = ntasks - 1 - gw - (q >> 2) * nw;
+        const int64_t band = t / strips, strip = t - band * strips;
+        const int g = (int)(q & 3);
+        const uint32_t stage = (uint32_t)(q % kTmaStages);
+        if (!q_mbar_wait(bar + 8 * stage, (uint32_t)((q / kTmaStages) & 1), kTmaWaitNs)) break;
+        uint2 raw[16];
+        const uint32_t src = ring + stage * kTmaStageBytes + (uint32_t)lane * 8u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(raw[i].x), "=r"(raw[i].y) : "r"(src + 256u * i));
+        // every lane's reads of the stage ordered before the async-proxy refill
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0 && q + kTmaStages < ngroups) issue(q + kTmaStages);
+        if (RHT) {  // the sign diagonal, on the packed rows
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                raw[i].x ^= sign_mask<uint16_t>(signs, i);
+                raw[i].y ^= sign_mask<uint16_t>(signs, i);
+            }
+        }
+        const int64_t c = strip * kTmaCols + lane * 4;
+        const int64_t rg = band * 64 + g * 16;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t w = (j >> 1) ? raw[i].y : raw[i].x;
+                v[i] = (j & 1) ? bf16hi(w) : bf16lo(w);
+            }
+            float scale_in;
+            uint32_t sb;
+            uint64_t pv[8];
+            float m = 0.0f;
+            if (RHT) {
+                fwht16_x2(v, pv);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m = fmaxf(m, fmaxf(fabsf(f2lo(pv[k])), fabsf(f2hi(pv[k]))));
+                sb = block_scale_code(__fmul_rn(m, 0.25f), ctx);  // max |z/4| = RN(max|z| / 4)
+                if (fold) {
+                    scale_in = s_inv4[sb];
+                } else {
+                    const uint64_t quarter = f2(0.25f, 0.25f);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) pv[k] = mul2_rn(pv[k], quarter);
+                    scale_in = s_inv[sb];
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    pv[k] = f2(v[2 * k], v[2 * k + 1]);
+                    m = fmaxf(m, fmaxf(fabsf(v[2 * k]), fabsf(v[2 * k + 1])));
+                }
+                sb = block_scale_code(m, ctx);
+                scale_in = s_inv[sb];
+            }
+            uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+            if (SR) sr_words16((uint64_t)(c + j) * (uint64_t)K + (uint64_t)rg, keys, w0, w1);  // rg % 16 == 0
+            stg[(g * 4 + j) * 32 + lane] = encode16_x2<SR>(pv, scale_in, w0, w1);
+            const int orow = lane * 4 + j;  // output row within the strip
+            atom[(orow & 31) * 16 + ((orow >> 5) & 3) * 4 + g] = (uint8_t)sb;
+        }
+        if (g == 3) {  // the task is complete: its 128 code rows and its scale atom
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t orow = c + j;
+                const int64_t room = K / 2 - band * 32;  // this band's code bytes in a row: 8, 16, 24 or 32
+                if (orow < p.C && NVFP4_IN_RANGE(orow * (K / 2) + band * 32, room < 32 ? room : 32, p.C * (K / 2))) {
+                    uint8_t *dst = p.codes + orow * (K / 2) + band * 32;
+                    const uint2 a0 = stg[(0 * 4 + j) * 32 + lane], a1 = stg[(1 * 4 + j) * 32 + lane];
+                    const uint2 a2 = stg[(2 * 4 + j) * 32 + lane], a3 = stg[(3 * 4 + j) * 32 + lane];
+                    if (room >= 32 && vec16) {
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+                        *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(a2.x, a2.y, a3.x, a3.y);
+                    } else {  // rows only 8-byte aligned (K % 32 == 16), or the last band
+                        *reinterpret_cast<uint2 *>(dst) = a0;
+                        if (room >= 16) *reinterpret_cast<uint2 *>(dst + 8) = a1;
+                        if (room >= 24) *reinterpret_cast<uint2 *>(dst + 16) = a2;
+                        if (room >= 32) *reinterpret_cast<uint2 *>(dst + 24) = a3;
+                    }
+                }
+            }
+            if (NVFP4_IN_RANGE((strip * KB4 + band) * 512 + lane * 16, 16, nv_scales_extent(p.C, K)))
+                *reinterpret_cast<uint4 *>(p.scales + (strip * KB4 + band) * 512 + lane * 16) =
+                    *reinterpret_cast<const uint4 *>(atom + lane * 16);
+            __syncwarp();
+        }
+    }
+    if (q < ngroups) {  // a load did not arrive in time: report, then let the loads in flight land
+        if (lane == 0 && p.status) atomicExch(p.status, 7);  // NVFP4_ERR_DEVICE_TIMEOUT
+        for (int64_t r = q; r < q + kTmaStages && r < ngroups; ++r)
+            q_mbar_wait(bar + 8 * (uint32_t)(r % kTmaStages), (uint32_t)((r / kTmaStages) & 1), kTmaDrainNs);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // MXFP4, rowwise, one pass (no tensor scale): blocks of 32 along the columns,
 // E8M0 scale 2^X with X = floor(log2 amax_b) - 2 clamped to [-127, 127], each
 // element E2M1(v * 2^-X) by round-to-nearest-even.  Same persistent walk and
@@ -805,6 +1024,57 @@ __global__ void tensor_scale_only_kernel(const float *amax_in, float *tensor_sca
     *tensor_scale = tensor_scale_from_amax(amax_in ? *amax_in : 0.0f);
 }
 
+// The driver's tensor-map encoder (looked up once).
+PFN_cuTensorMapEncodeTiled_v12000 q_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// bf16 input [R x C] (leading dimension ld) as 16-row x 128-column boxes; outside
+// the tensor a box reads zeros.
+bool make_colwise_map(CUtensorMap *map, const void *x, int64_t R, int64_t C, int64_t ld) {
+    auto fn = q_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)R};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)kTmaCols, 16u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool SR, bool RHT>
+cudaError_t launch_colwise_tma(const QParams &p, cudaStream_t s) {
+    CUtensorMap map;
+    if (!make_colwise_map(&map, p.x, p.R, p.C, p.ld)) return cudaErrorInvalidValue;
+    constexpr int kMaxDev = 64;
+    static bool attr_set[kMaxDev] = {};  // per instantiation and device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(quantize_colwise_tma_kernel<SR, RHT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tma_smem_bytes<SR>());
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int64_t ntasks = ((p.C + kTmaCols - 1) / kTmaCols) * ((p.R + 63) / 64);
+    const unsigned grid =
+        (unsigned)std::min<int64_t>((ntasks + kTmaWarps - 1) / kTmaWarps, tma_ctas<SR>() * (int64_t)num_sms());
+    quantize_colwise_tma_kernel<SR, RHT><<<grid, 32 * kTmaWarps, tma_smem_bytes<SR>(), s>>>(map, p);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
     const T *x = static_cast<const T *>(a.x);
@@ -829,6 +1099,7 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
     QParams p{a.x, a.R, a.C, a.ld, a.seed, a.amax_in, a.partials, num_partials, a.codes, a.scales,
               a.tensor_scale};
     p.aligned32 = (reinterpret_cast<uintptr_t>(a.x) % 32 == 0) && ((a.ld * (int64_t)sizeof(T)) % 32 == 0);
+    p.status = a.status;
     constexpr int N = Vec<T>::N;  // columns per lane of the colwise kernels
     if (!a.colwise) {
         constexpr int tile_r = sizeof(T) == 2 ? 32 : 16;  // rows per tile of quantize_rowwise_kernel
@@ -836,6 +1107,13 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
         const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
         if (a.sr) quantize_rowwise_kernel<T, true><<<grid, kThreads, 0, s>>>(p);
         else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);
+    } else if (sizeof(T) == 2) {  // bf16: the TMA-fed colwise kernel
+        cudaError_t e;
+        if (a.sr && a.rht) e = launch_colwise_tma<true, true>(p, s);
+        else if (a.sr) e = launch_colwise_tma<true, false>(p, s);
+        else if (a.rht) e = launch_colwise_tma<false, true>(p, s);
+        else e = launch_colwise_tma<false, false>(p, s);
+        if (e != cudaSuccess) return e;
     } else {
         dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 255) / 256));
         if (a.sr && a.rht) quantize_colwise_kernel<T, true, true, false><<<grid, kThreads, 0, s>>>(p);
