@@ -84,6 +84,29 @@ typedef struct nvfp4_tensor {
     int64_t k;
 } nvfp4_tensor;
 
+/*
+ * nvfp4_amax -- the tensor amax of the FP32 per-tensor scale (aisight.pl,
+ * section "Architektura NVFP4 kontra ograniczenia mikroskalowania": one FP32
+ * scale per tensor next to the E4M3 block scales): *amax_out = max |x| over the
+ * [R x C] tensor x (leading dimension ld elements), or with rht = 1 the max of
+ * |y| over y = 1/4 H16 D v, the random Hadamard transform applied down every
+ * 16-row group of every column as the colwise quantisation of the Wgrad
+ * operands applies it (same page, section "Technologie stabilizujace proces
+ * treningowy"; signs D from `seed`).  Exactly the amax nvfp4_quantize computes
+ * in its first pass, so handing it on as amax_in gives the same codes; one
+ * amax serves both orientations of a tensor without the transform.  An empty
+ * tensor gives 0.  amax_out: device memory, one float, caller-owned;
+ * workspace: >= nvfp4_quantize_workspace_size() bytes, 16-byte aligned
+ * (per-CTA partials).  Requires x 16-byte aligned, ld * element size and
+ * C * element size multiples of 16, R % 16 == 0 when rht, R, C <= 2^31.
+ * Asynchronous (two launches).  Errors: NVFP4_ERR_INVALID_ARG, NVFP4_ERR_SHAPE,
+ * NVFP4_ERR_ALIGNMENT, NVFP4_ERR_WORKSPACE, NVFP4_ERR_UNSUPPORTED_DEVICE,
+ * NVFP4_ERR_CUDA.
+ */
+NVFP4_API nvfp4_status nvfp4_amax(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, int rht,
+                                  uint64_t seed, float *amax_out, void *workspace, size_t ws_bytes,
+                                  cudaStream_t stream);
+
 /* Sizes of the two byte buffers of an NVFP4 tensor (k must be a multiple of 16). */
 NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t k);
 NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t k);

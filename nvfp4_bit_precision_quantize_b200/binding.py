@@ -41,7 +41,7 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
            "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
            "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd", "nvfp4_selftest_mma_rate",
-           "nvfp4_bounds_status", "nvfp4_selftest_bounds")
+           "nvfp4_bounds_status", "nvfp4_selftest_bounds", "nvfp4_amax")
 
 
 class CTensor(C.Structure):
@@ -90,6 +90,7 @@ def load():
         "nvfp4_selftest_wait_timeout": (i32, [vp, sz, u64, vp]),
         "nvfp4_selftest_mma_rate": (i32, [i32, i64, vp, i64, C.POINTER(C.c_int), vp, sz, vp]),
         "nvfp4_bounds_status": (i32, [C.POINTER(C.c_int), C.POINTER(C.c_int)]),
+        "nvfp4_amax": (i32, [vp, i32, i64, i64, i64, i32, u64, vp, vp, sz, vp]),
         "nvfp4_selftest_bounds": (i32, [vp, i64, vp]),
         "nvfp4_quantize_dual_workspace_size": (sz, []),
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
@@ -264,6 +265,19 @@ def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, 
                                int(bool(rht)), seed, _ptr(amax_in), C.byref(ct), _ptr(ws), _workspace(ws),
                                _stream(stream))
     _ok(st, "nvfp4_quantize")
+    return out
+
+
+def nvfp4_amax(x, rht=False, seed=1234, out=None, ws=None, stream=None):
+    """max |x| of a 2-D float32/bfloat16 CUDA tensor (with rht, of the 16-row Hadamard transform of
+    its columns) into a one-float device tensor, as nvfp4_quantize's amax pass computes it."""
+    _rows("x", x)
+    R, Cc = x.shape
+    out = _amax_buffer(out, x.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_workspace_size(), x.device)
+    _on_device(x, out, ws)
+    _ok(load().nvfp4_amax(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), int(bool(rht)), seed, _ptr(out),
+                          _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_amax")
     return out
 
 

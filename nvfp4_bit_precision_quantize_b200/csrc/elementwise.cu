@@ -213,6 +213,12 @@ cudaError_t launch_relu2_amax_rht(const void *dh, const void *y, void *out, int6
     return cudaGetLastError();
 }
 
+cudaError_t launch_amax_reduce(const float *partials, int count, float *amax_out, cudaStream_t s, int *launches) {
+    amax_reduce_kernel<<<1, kThreads, 0, s>>>(partials, count, amax_out);
+    ++*launches;
+    return cudaGetLastError();
+}
+
 cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_out, float *amax_rht_out, cudaStream_t s,
                                 int *launches) {
     amax_reduce2_kernel<<<1, kThreads, 0, s>>>(partials, partials + kMaxPartials, count, amax_out, amax_rht_out);

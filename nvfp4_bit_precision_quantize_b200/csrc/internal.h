@@ -84,6 +84,10 @@ cudaError_t launch_relu2_bwd(const void *dh, const void *y, void *dy, int64_t n,
                              cudaStream_t s, int *launches);
 
 // max over per-CTA partials (plain at partials, RHT at partials + kMaxPartials) -> *amax_out, *amax_rht_out
+cudaError_t launch_amax_reduce(const float *partials, int count, float *amax_out, cudaStream_t s, int *launches);
+// Tensor amax (after the 16-row RHT when rht): per-CTA partials, then one reduce into *amax_out.
+cudaError_t launch_amax(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool rht, uint64_t seed,
+                        float *partials, float *amax_out, cudaStream_t s, int *launches);
 cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_out, float *amax_rht_out, cudaStream_t s,
                                 int *launches);
 

@@ -1162,6 +1162,37 @@ cudaError_t run_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches) {
 
 }  // namespace
 
+namespace {
+template <typename T>
+cudaError_t run_amax(const T *x, int64_t R, int64_t C, int64_t ld, bool rht, uint64_t seed, float *partials,
+                     float *amax_out, cudaStream_t s, int *launches) {
+    const int sms = num_sms();
+    int n;
+    if (rht) {
+        const int64_t units = (R / 16) * (C / Vec<T>::N);
+        n = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                   std::max<int64_t>(1, (units + kThreads - 1) / kThreads));
+        amax_rht_kernel<T><<<n, kThreads, 0, s>>>(x, R, C, ld, seed, partials);
+    } else {
+        const int64_t chunks = R * (C / Vec<T>::N);
+        n = (int)std::min<int64_t>(std::min<int64_t>(4 * sms, kMaxPartials),
+                                   std::max<int64_t>(1, (chunks + kThreads - 1) / kThreads));
+        amax_kernel<T><<<n, kThreads, 0, s>>>(x, R, C, ld, partials);
+    }
+    ++*launches;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_amax_reduce(partials, n, amax_out, s, launches);
+}
+}  // namespace
+
+cudaError_t launch_amax(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool rht, uint64_t seed,
+                        float *partials, float *amax_out, cudaStream_t s, int *launches) {
+    if (R == 0 || C == 0) return cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    return bf16 ? run_amax(static_cast<const uint16_t *>(x), R, C, ld, rht, seed, partials, amax_out, s, launches)
+                : run_amax(static_cast<const float *>(x), R, C, ld, rht, seed, partials, amax_out, s, launches);
+}
+
 cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int *launches) {
     if (a.R == 0 || a.C == 0) {
         tensor_scale_only_kernel<<<1, 1, 0, s>>>(a.amax_row_in, a.row_tensor_scale);

@@ -10,10 +10,11 @@ treningowy").  This module only orders the calls and holds the buffers:
 argument marshalling through `binding`, all arithmetic in the CUDA library.
 
 A step, with X [M x H], W1 [F x H], W2 [H x F], dY2 [M x H] (bf16):
-  forward   X_r = rowwise(X); W1_r, W1_c = dual(W1)
+  forward   X_r = rowwise(X); a1 = amax(W1); W1_r = rowwise(W1, a1); W1_c = colwise(W1, a1)
             Y1 = X_r . W1_r^T and h = relu(Y1)^2 from one GEMM (the epilogue also
             returns max|h| and max|RHT(h)|)
-            h_r = rowwise(h, amax supplied); W2_r, W2_c = dual(W2); Y2 = h_r . W2_r^T
+            h_r = rowwise(h, amax supplied); a2 = amax(W2); W2_r = rowwise(W2, a2);
+            W2_c = colwise(W2, a2); Y2 = h_r . W2_r^T
   backward  dY2_r = rowwise(dY2)
             dY1 = (dY2_r . W2_c^T) * 2 relu(Y1) from one GEMM (the epilogue applies the
             derivative to the bf16 dh, which is never stored, and returns max|dY1| and
@@ -59,6 +60,7 @@ class MlpStep:
         self.ws = B.workspace(256, device)      # GEMM status word
         self.qws = B.workspace(B.nvfp4_quantize_dual_workspace_size(), device)
         self.amax = torch.zeros(16, dtype=torch.float32, device=device)  # h, RHT(h), dY1, RHT(dY1) at 0, 4, 8, 12
+        self.wamax = torch.zeros(8, dtype=torch.float32, device=device)  # W1, W2 at 0, 4
         mk = B.empty_nvfp4
         self.q = {
             "X_r": mk(M, H, device), "W1_r": mk(F, H, device), "W1_c": mk(H, F, device),
@@ -83,11 +85,13 @@ class MlpStep:
                          out=self.q[key], ws=self.qws)
         self._mark(ev, "quant", x.numel() * bytes_per_elem(amax_in is not None) if bytes_per_elem else 0)
 
-    def _dual(self, x, key_r, key_c, sr=False, rht=False, ev=None, bytes_per_elem=None):
-        B = self.B
-        B.nvfp4_quantize_dual(x, col_rounding=B.NVFP4_SR if sr else B.NVFP4_RTN, col_rht=rht, seed=self.seed,
-                              out_row=self.q[key_r], out_col=self.q[key_c], ws=self.qws)
-        self._mark(ev, "quant", x.numel() * bytes_per_elem("dual") if bytes_per_elem else 0)
+    def _weight(self, w, key_r, key_c, amax, ev=None, bytes_per_elem=None):
+        """A weight's two RTN operands from one amax pass: the amax does not depend on the
+        orientation (no transform), so both quantisations take it as supplied."""
+        self.B.nvfp4_amax(w, out=amax, ws=self.qws)
+        self._mark(ev, "quant", w.numel() * bytes_per_elem("amax") if bytes_per_elem else 0)
+        self._quant(w, key_r, amax_in=amax, ev=ev, bytes_per_elem=bytes_per_elem)
+        self._quant(w, key_c, colwise=True, amax_in=amax, ev=ev, bytes_per_elem=bytes_per_elem)
 
     def _gemm(self, a, b, out, ev=None):
         self.B.nvfp4_gemm(self.q[a], self.q[b], out=out, ws=self.ws)
@@ -98,7 +102,7 @@ class MlpStep:
         Y2 = self.Y2 if Y2 is None else Y2
         kw = dict(ev=ev, bytes_per_elem=bytes_per_elem)
         self._quant(X, "X_r", **kw)
-        self._dual(d["W1"], "W1_r", "W1_c", **kw)
+        self._weight(d["W1"], "W1_r", "W1_c", self.wamax[0:1], **kw)
         # relu^2 also returns max|h| and max|RHT(h)|: both quantisations of h skip their amax pass
         if self.fused:
             self.B.nvfp4_gemm_relu2_fwd(self.q["X_r"], self.q["W1_r"], seed=self.seed, y=self.Y1, h=self.h,
@@ -110,7 +114,7 @@ class MlpStep:
                                             amax_rht_out=self.amax[4:5], ws=self.qws)
             self._mark(ev, "relu2", self.Y1.numel())
         self._quant(self.h, "h_r", amax_in=self.amax[0:1], **kw)
-        self._dual(d["W2"], "W2_r", "W2_c", **kw)
+        self._weight(d["W2"], "W2_r", "W2_c", self.wamax[4:5], **kw)
         self._gemm("h_r", "W2_r", Y2, ev)
 
     def backward(self, X=None, dY2=None, ev=None, bytes_per_elem=None, grad_ready=None):

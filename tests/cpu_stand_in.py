@@ -69,6 +69,12 @@ def nvfp4_quantize(x, orientation=NVFP4_ROWWISE, rounding=NVFP4_RTN, rht=False, 
     return out
 
 
+def nvfp4_amax(x, rht=False, seed=1234, out=None, ws=None):
+    calls.append("amax")
+    out.fill_(float(oracle.amax(_bits(x), colwise=bool(rht), rht=bool(rht), seed=seed)))
+    return out
+
+
 def nvfp4_quantize_dual(x, col_rounding=NVFP4_RTN, col_rht=False, seed=1234, out_row=None, out_col=None, ws=None):
     calls.append("quantize_dual")
     b = _bits(x)

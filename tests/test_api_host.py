@@ -183,6 +183,27 @@ def test_selftest_rejections(lib):
     assert lib.nvfp4_selftest_wait_timeout(ws, 256, 3_000_000_000, None) == binding.NVFP4_ERR_INVALID_ARG
 
 
+def test_amax_rejections(lib):
+    f = lib.nvfp4_amax
+    f.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_int, C.c_uint64, C.c_void_p, C.c_void_p,
+                  C.c_size_t, C.c_void_p]
+    E, bf = binding, binding.NVFP4_DTYPE_BF16
+    x, out, ws = C.c_void_p(0x10000), C.c_void_p(0x30000), C.c_void_p(0x40000)
+    wsb = lib.nvfp4_quantize_workspace_size()
+    assert f(x, bf, 64, 64, 64, 0, 1, None, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG        # no output
+    assert f(x, 7, 64, 64, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG          # dtype
+    assert f(x, bf, 64, 64, 64, 2, 1, out, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG         # rht flag
+    assert f(x, bf, 64, 64, 64, 0, 1, C.c_void_p(0x30002), ws, wsb, None) == E.NVFP4_ERR_ALIGNMENT
+    assert f(x, bf, -1, 64, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_SHAPE
+    assert f(x, bf, 64, 64, 64, 0, 1, out, None, wsb, None) == E.NVFP4_ERR_WORKSPACE
+    assert f(x, bf, 64, 64, 64, 0, 1, out, ws, wsb - 1, None) == E.NVFP4_ERR_WORKSPACE
+    assert f(None, bf, 64, 64, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG      # no input
+    assert f(x, bf, 64, 60, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_SHAPE               # C * 2 % 16
+    assert f(x, bf, 40, 64, 64, 1, 1, out, ws, wsb, None) == E.NVFP4_ERR_SHAPE               # rht: R % 16
+    assert f(x, bf, 64, 64, 32, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_SHAPE               # ld < C
+    assert f(C.c_void_p(0x10008), bf, 64, 64, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_ALIGNMENT
+
+
 def test_mma_rate_probe_rejections(lib):
     ws, cyc, pairs = C.c_void_p(0x20000), C.c_void_p(0x40000), C.c_int(0)
     f = lib.nvfp4_selftest_mma_rate

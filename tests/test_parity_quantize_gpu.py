@@ -2,11 +2,12 @@
 padding, FP32 tensor scale), through the C ABI."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from nvfp4_bit_precision_quantize_b200 import workloads as W
 
-from gpu_helpers import check_quantize, gpu_quantize, f32_bits, first_mismatch
+from gpu_helpers import check_quantize, gpu_quantize, f32_bits, first_mismatch, to_dev
 import layout
 
 pytestmark = pytest.mark.gpu
@@ -136,3 +137,29 @@ def test_wgrad_operands_full_size(cuda_lib):
     w = W.wgrad()
     _sampled_check(w["dY"], True, True, True, seed=1234, n_rows=24)
     _sampled_check(w["X"], True, False, True, seed=1234, n_rows=24)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rht", [False, True], ids=["plain", "rht"])
+def test_amax_matches_oracle(dtype, rht, cuda_lib):
+    """nvfp4_amax: the tensor amax (after the 16-row RHT when asked) bit-exact against the
+    oracle's, on ragged shapes and at a full weight shape; the quantisations it feeds give the
+    same codes as their own amax pass (aisight.pl, sections "Architektura NVFP4 kontra
+    ograniczenia mikroskalowania" and "Technologie stabilizujace proces treningowy")."""
+    B = cuda_lib
+    rng = np.random.default_rng(17)
+    for R, C in [(16, 16), (48, 272), (528, 64), (1024, 1040)]:
+        x = W.normal(rng, (R, C), 0.5)
+        xb = W.bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
+        got = B.nvfp4_amax(to_dev(xb), rht=rht, seed=1234)
+        want = oracle.amax(xb, colwise=rht, rht=rht, seed=1234)
+        assert f32_bits(got.cpu().numpy()[0]) == f32_bits(np.float32(want)), (R, C)
+    x = to_dev(W.bf16_bits(W.normal(rng, (5120, 2048), 0.02)))
+    ws = B.workspace(B.nvfp4_quantize_workspace_size(), x.device)
+    a = B.nvfp4_amax(x, ws=ws)
+    for orient in (B.NVFP4_ROWWISE, B.NVFP4_COLWISE):
+        q0 = B.nvfp4_quantize(x, orientation=orient, ws=ws)
+        q1 = B.nvfp4_quantize(x, orientation=orient, amax_in=a, ws=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(q0.codes, q1.codes) and torch.equal(q0.scales, q1.scales)
+        assert torch.equal(q0.tensor_scale, q1.tensor_scale)
