@@ -107,6 +107,20 @@ NVFP4_API nvfp4_status nvfp4_amax(const void *x, nvfp4_dtype dtype, int64_t R, i
                                   uint64_t seed, float *amax_out, void *workspace, size_t ws_bytes,
                                   cudaStream_t stream);
 
+/*
+ * nvfp4_amax_dual -- both amaxes of a tensor whose rowwise and colwise-RHT
+ * operands are both needed (the Fprop and Wgrad operands of one activation or
+ * gradient), from one read: *amax_out = max |x| and *amax_rht_out = max |y|,
+ * y = 1/4 H16 D v down every 16-row group of every column, bit for bit what
+ * nvfp4_amax gives with rht = 0 and 1 (same passages).  amax_out, amax_rht_out:
+ * device memory, one float each; workspace: >= nvfp4_quantize_dual_workspace_size()
+ * bytes, 16-byte aligned.  Requires R % 16 == 0 and the rest as nvfp4_amax.
+ * Asynchronous (two launches).  Errors as nvfp4_amax.
+ */
+NVFP4_API nvfp4_status nvfp4_amax_dual(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld,
+                                       uint64_t seed, float *amax_out, float *amax_rht_out, void *workspace,
+                                       size_t ws_bytes, cudaStream_t stream);
+
 /* Sizes of the two byte buffers of an NVFP4 tensor (k must be a multiple of 16). */
 NVFP4_API size_t nvfp4_codes_bytes(int64_t rows, int64_t k);
 NVFP4_API size_t nvfp4_scales_bytes(int64_t rows, int64_t k);

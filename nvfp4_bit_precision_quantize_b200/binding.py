@@ -41,7 +41,8 @@ EXPORTS = ("nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_quantize_workspace_
            "nvfp4_relu2_bwd_amax", "nvfp4_mx_scales_bytes", "nvfp4_quantize_mx",
            "nvfp4_relu2_fwd_amax_rht", "nvfp4_relu2_bwd_amax_rht", "nvfp4_linear_fwd_workspace_size",
            "nvfp4_gemm_mx", "nvfp4_gemm_relu2_fwd", "nvfp4_gemm_relu2_bwd", "nvfp4_selftest_mma_rate",
-           "nvfp4_bounds_status", "nvfp4_selftest_bounds", "nvfp4_amax")
+           "nvfp4_bounds_status", "nvfp4_selftest_bounds", "nvfp4_amax",
+           "nvfp4_amax_dual")
 
 
 class CTensor(C.Structure):
@@ -91,6 +92,7 @@ def load():
         "nvfp4_selftest_mma_rate": (i32, [i32, i64, vp, i64, C.POINTER(C.c_int), vp, sz, vp]),
         "nvfp4_bounds_status": (i32, [C.POINTER(C.c_int), C.POINTER(C.c_int)]),
         "nvfp4_amax": (i32, [vp, i32, i64, i64, i64, i32, u64, vp, vp, sz, vp]),
+        "nvfp4_amax_dual": (i32, [vp, i32, i64, i64, i64, u64, vp, vp, vp, sz, vp]),
         "nvfp4_selftest_bounds": (i32, [vp, i64, vp]),
         "nvfp4_quantize_dual_workspace_size": (sz, []),
         "nvfp4_quantize_dual": (i32, [vp, i32, i64, i64, i64, i32, i32, u64, vp, vp, tp, tp, vp, sz, vp]),
@@ -279,6 +281,20 @@ def nvfp4_amax(x, rht=False, seed=1234, out=None, ws=None, stream=None):
     _ok(load().nvfp4_amax(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), int(bool(rht)), seed, _ptr(out),
                           _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_amax")
     return out
+
+
+def nvfp4_amax_dual(x, seed=1234, out=None, out_rht=None, ws=None, stream=None):
+    """max |x| and max |RHT(x)| (16-row transform down the columns) of a 2-D float32/bfloat16 CUDA
+    tensor from one read; returns the two one-float device tensors."""
+    _rows("x", x)
+    R, Cc = x.shape
+    out = _amax_buffer(out, x.device)
+    out_rht = _amax_buffer(out_rht, x.device)
+    ws = ws if ws is not None else workspace(nvfp4_quantize_dual_workspace_size(), x.device)
+    _on_device(x, out, out_rht, ws)
+    _ok(load().nvfp4_amax_dual(_ptr(x), _dtype_code(x.dtype), R, Cc, x.stride(0), seed, _ptr(out), _ptr(out_rht),
+                               _ptr(ws), _workspace(ws), _stream(stream)), "nvfp4_amax_dual")
+    return out, out_rht
 
 
 def nvfp4_mx_scales_bytes(rows, k):

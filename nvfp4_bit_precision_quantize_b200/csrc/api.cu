@@ -331,6 +331,29 @@ nvfp4_status nvfp4_amax(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, 
                                            stream, &call.launches)));
 }
 
+nvfp4_status nvfp4_amax_dual(const void *x, nvfp4_dtype dtype, int64_t R, int64_t C, int64_t ld, uint64_t seed,
+                             float *amax_out, float *amax_rht_out, void *workspace, size_t ws_bytes,
+                             cudaStream_t stream) {
+    Call call(__func__);
+    if (!amax_out || !amax_rht_out || !valid_dtype(dtype)) return NVFP4_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(amax_out) % 4 != 0 || reinterpret_cast<uintptr_t>(amax_rht_out) % 4 != 0)
+        return NVFP4_ERR_ALIGNMENT;
+    if (R < 0 || C < 0 || R > (1LL << 31) || C > (1LL << 31)) return NVFP4_ERR_SHAPE;
+    if (!workspace || ws_bytes < kDualWorkspace) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+    const size_t es = esize(dtype);
+    if (R > 0 && C > 0) {
+        if (!x) return NVFP4_ERR_INVALID_ARG;
+        if (ld < C || (C * (int64_t)es) % 16 != 0 || R % 16 != 0) return NVFP4_ERR_SHAPE;
+        if (!aligned16(x) || (ld * (int64_t)es) % 16 != 0) return NVFP4_ERR_ALIGNMENT;
+    }
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    float *partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    return call.done(from_cuda(launch_amax_dual(x, dtype == NVFP4_DTYPE_BF16, R, C, ld, seed, partials, amax_out,
+                                                amax_rht_out, stream, &call.launches)));
+}
+
 size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;
     return (size_t)((rows + 127) / 128) * 128 * (size_t)((k + 127) / 128) * 4;

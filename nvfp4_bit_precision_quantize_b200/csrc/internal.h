@@ -88,6 +88,9 @@ cudaError_t launch_amax_reduce(const float *partials, int count, float *amax_out
 // Tensor amax (after the 16-row RHT when rht): per-CTA partials, then one reduce into *amax_out.
 cudaError_t launch_amax(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool rht, uint64_t seed,
                         float *partials, float *amax_out, cudaStream_t s, int *launches);
+// Both amaxes (plain and after the 16-row RHT) from one read: partials (2 x kMaxPartials), then one reduce.
+cudaError_t launch_amax_dual(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, uint64_t seed,
+                             float *partials, float *amax_out, float *amax_rht_out, cudaStream_t s, int *launches);
 cudaError_t launch_amax_reduce2(const float *partials, int count, float *amax_out, float *amax_rht_out, cudaStream_t s,
                                 int *launches);
 

@@ -1186,6 +1186,33 @@ cudaError_t run_amax(const T *x, int64_t R, int64_t C, int64_t ld, bool rht, uin
 }
 }  // namespace
 
+namespace {
+template <typename T>
+cudaError_t run_amax_dual(const T *x, int64_t R, int64_t C, int64_t ld, uint64_t seed, float *partials,
+                          float *amax_out, float *amax_rht_out, cudaStream_t s, int *launches) {
+    const int64_t units = (R / 16) * (C / Vec<T>::N);
+    const int n = (int)std::min<int64_t>(std::min<int64_t>(4 * num_sms(), kMaxPartials),
+                                         std::max<int64_t>(1, (units + kThreads - 1) / kThreads));
+    amax_dual_kernel<T><<<n, kThreads, 0, s>>>(x, R, C, ld, seed, partials, partials + kMaxPartials);
+    ++*launches;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_amax_reduce2(partials, n, amax_out, amax_rht_out, s, launches);
+}
+}  // namespace
+
+cudaError_t launch_amax_dual(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, uint64_t seed,
+                             float *partials, float *amax_out, float *amax_rht_out, cudaStream_t s, int *launches) {
+    if (R == 0 || C == 0) {
+        cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+        return e != cudaSuccess ? e : cudaMemsetAsync(amax_rht_out, 0, sizeof(float), s);
+    }
+    return bf16 ? run_amax_dual(static_cast<const uint16_t *>(x), R, C, ld, seed, partials, amax_out, amax_rht_out,
+                                s, launches)
+                : run_amax_dual(static_cast<const float *>(x), R, C, ld, seed, partials, amax_out, amax_rht_out, s,
+                                launches);
+}
+
 cudaError_t launch_amax(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool rht, uint64_t seed,
                         float *partials, float *amax_out, cudaStream_t s, int *launches) {
     if (R == 0 || C == 0) return cudaMemsetAsync(amax_out, 0, sizeof(float), s);

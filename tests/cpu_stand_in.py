@@ -75,6 +75,14 @@ def nvfp4_amax(x, rht=False, seed=1234, out=None, ws=None):
     return out
 
 
+def nvfp4_amax_dual(x, seed=1234, out=None, out_rht=None, ws=None):
+    calls.append("amax_dual")
+    b = _bits(x)
+    out.fill_(float(oracle.amax(b)))
+    out_rht.fill_(float(oracle.amax(b, colwise=True, rht=True, seed=seed)))
+    return out, out_rht
+
+
 def nvfp4_quantize_dual(x, col_rounding=NVFP4_RTN, col_rht=False, seed=1234, out_row=None, out_col=None, ws=None):
     calls.append("quantize_dual")
     b = _bits(x)

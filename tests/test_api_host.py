@@ -204,6 +204,22 @@ def test_amax_rejections(lib):
     assert f(C.c_void_p(0x10008), bf, 64, 64, 64, 0, 1, out, ws, wsb, None) == E.NVFP4_ERR_ALIGNMENT
 
 
+def test_amax_dual_rejections(lib):
+    f = lib.nvfp4_amax_dual
+    f.argtypes = [C.c_void_p, C.c_int, C.c_int64, C.c_int64, C.c_int64, C.c_uint64, C.c_void_p, C.c_void_p,
+                  C.c_void_p, C.c_size_t, C.c_void_p]
+    E, bf = binding, binding.NVFP4_DTYPE_BF16
+    x, o1, o2, ws = C.c_void_p(0x10000), C.c_void_p(0x30000), C.c_void_p(0x30010), C.c_void_p(0x40000)
+    wsb = lib.nvfp4_quantize_dual_workspace_size()
+    assert f(x, bf, 64, 64, 64, 1, None, o2, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG
+    assert f(x, bf, 64, 64, 64, 1, o1, None, ws, wsb, None) == E.NVFP4_ERR_INVALID_ARG
+    assert f(x, bf, 64, 64, 64, 1, o1, C.c_void_p(0x30011), ws, wsb, None) == E.NVFP4_ERR_ALIGNMENT
+    assert f(x, bf, 64, 64, 64, 1, o1, o2, ws, lib.nvfp4_quantize_workspace_size(), None) == E.NVFP4_ERR_WORKSPACE
+    assert f(x, bf, 40, 64, 64, 1, o1, o2, ws, wsb, None) == E.NVFP4_ERR_SHAPE               # R % 16
+    assert f(x, bf, 64, 60, 64, 1, o1, o2, ws, wsb, None) == E.NVFP4_ERR_SHAPE               # C * 2 % 16
+    assert f(C.c_void_p(0x10008), bf, 64, 64, 64, 1, o1, o2, ws, wsb, None) == E.NVFP4_ERR_ALIGNMENT
+
+
 def test_mma_rate_probe_rejections(lib):
     ws, cyc, pairs = C.c_void_p(0x20000), C.c_void_p(0x40000), C.c_int(0)
     f = lib.nvfp4_selftest_mma_rate

@@ -163,3 +163,17 @@ def test_amax_matches_oracle(dtype, rht, cuda_lib):
         torch.cuda.synchronize()
         assert torch.equal(q0.codes, q1.codes) and torch.equal(q0.scales, q1.scales)
         assert torch.equal(q0.tensor_scale, q1.tensor_scale)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_amax_dual_matches_oracle(dtype, cuda_lib):
+    """nvfp4_amax_dual: both amaxes from one read, each bit-exact against the oracle's (the same
+    passages as nvfp4_amax)."""
+    B = cuda_lib
+    rng = np.random.default_rng(19)
+    for R, C in [(16, 16), (48, 272), (528, 64), (1024, 1040)]:
+        x = W.normal(rng, (R, C), 0.5)
+        xb = W.bf16_bits(x) if dtype == "bf16" else x.astype(np.float32)
+        a, b = B.nvfp4_amax_dual(to_dev(xb), seed=99)
+        assert f32_bits(a.cpu().numpy()[0]) == f32_bits(oracle.amax(xb)), (R, C)
+        assert f32_bits(b.cpu().numpy()[0]) == f32_bits(oracle.amax(xb, colwise=True, rht=True, seed=99)), (R, C)
