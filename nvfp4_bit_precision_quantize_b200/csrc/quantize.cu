@@ -424,8 +424,9 @@ __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_kernel(const QPa
 }
 
 // ---------------------------------------------------------------------------
-// Pass 2, colwise: blocks of 16 run down the rows; the output is the transpose
-// ([C x R], K = R contiguous).  CTA tile = 256 rows x (32*N) columns; warp w
+// Pass 2, colwise, register-fed (f32 input, and the dual pass for both dtypes;
+// bf16 single quantisations take quantize_colwise_tma_kernel below): blocks of
+// 16 run down the rows; the output is the transpose ([C x R], K = R contiguous).  CTA tile = 256 rows x (32*N) columns; warp w
 // owns rows 32w..32w+31 (two 16-row groups) and each lane N adjacent columns,
 // so every block (one column x 16 rows) sits in one thread's registers: the
 // transform, block amax and encoding need no shuffles.  The Hadamard signs
@@ -1107,14 +1108,14 @@ cudaError_t run(const QuantizeArgs &a, cudaStream_t s, int *launches) {
         const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
         if (a.sr) quantize_rowwise_kernel<T, true><<<grid, kThreads, 0, s>>>(p);
         else quantize_rowwise_kernel<T, false><<<grid, kThreads, 0, s>>>(p);
-    } else if (sizeof(T) == 2) {  // bf16: the TMA-fed colwise kernel
+    } else if constexpr (sizeof(T) == 2) {  // bf16: the TMA-fed colwise kernel
         cudaError_t e;
         if (a.sr && a.rht) e = launch_colwise_tma<true, true>(p, s);
         else if (a.sr) e = launch_colwise_tma<true, false>(p, s);
         else if (a.rht) e = launch_colwise_tma<false, true>(p, s);
         else e = launch_colwise_tma<false, false>(p, s);
         if (e != cudaSuccess) return e;
-    } else {
+    } else {  // f32 input: the register-fed colwise kernel
         dim3 grid((unsigned)((a.C + 32 * N - 1) / (32 * N)), (unsigned)((a.R + 255) / 256));
         if (a.sr && a.rht) quantize_colwise_kernel<T, true, true, false><<<grid, kThreads, 0, s>>>(p);
         else if (a.sr) quantize_colwise_kernel<T, true, false, false><<<grid, kThreads, 0, s>>>(p);
