@@ -861,15 +861,22 @@ __global__ void __launch_bounds__(32 * kTmaWarps, tma_ctas<SR>())
 // ---------------------------------------------------------------------------
 // MXFP4, rowwise, one pass (no tensor scale): blocks of 32 along the columns,
 // E8M0 scale 2^X with X = floor(log2 amax_b) - 2 clamped to [-127, 127], each
-// element E2M1(v * 2^-X) by round-to-nearest-even.  Same persistent walk and
-// 64-row tiles as the NVFP4 rowwise pass; a block spans 32/N lanes of a row.
-// Scales use the 128x4 atom order with four 32-blocks per atom word.
+// element E2M1(v * 2^-X) by round-to-nearest-even.  As in the NVFP4 rowwise
+// pass, each lane owns one whole block of a row (64 bytes of bf16, 128 of f32),
+// so the block amax, the E8M0 code and the 32 codes (one 16-byte store) need
+// no shuffles; a warp covers 1024 columns of RPW rows per tile, persistent CTAs
+// walk the tiles in reverse order with the next tile's loads in flight.  Scales
+// use the 128x4 atom order with four 32-blocks per atom word, a word held by
+// four neighbouring lanes: two shuffles gather it and one lane stores it.
+// Padding rows (to the atoms' 128-row extent) and padding blocks (to their
+// 4-block width) load zeros and get code 0.
 // ---------------------------------------------------------------------------
 struct MxParams {
     const void *x;
     int64_t R, C, ld;
     uint8_t *codes;
     uint8_t *scales;
+    int aligned32;  // x and every row start 32-byte aligned (256-bit loads allowed)
 };
 
 // E8M0 code of a block amax (finite, >= 0): the biased exponent field minus 2
@@ -881,85 +888,75 @@ __device__ __forceinline__ uint32_t mx_code(float amax) {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) quantize_rowwise_mx_kernel(const MxParams p) {
-    constexpr int N = Vec<T>::N;
-    constexpr int LPB = 32 / N;          // lanes per 32-block
-    constexpr int TILE_C = 32 * N;
-    constexpr int TILE_R = 64;
-    constexpr int RPW = TILE_R / (kThreads / 32);
-    constexpr int ATOMS = TILE_C / 128;  // scale atoms per tile row band
-    __shared__ __align__(16) uint8_t s_sc[ATOMS * 512];
-
+    constexpr int LW = 8 * (int)sizeof(T);          // 32-bit words per lane and row: 16 (bf16), 32 (f32)
+    constexpr int RPW = sizeof(T) == 2 ? 2 : 1;     // rows per warp per tile
+    constexpr int TILE_R = RPW * (kThreads / 32);
+    constexpr int TILE_B = 32;                      // blocks (of 32 columns) per tile row
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const T *x = static_cast<const T *>(p.x);
-    const int64_t K = p.C;
-    const int64_t KB4 = (K + 127) / 128;
-    const int64_t tiles_c = (p.C + TILE_C - 1) / TILE_C;
-    const int64_t tiles_r = 2 * ((p.R + 127) / 128);
+    const uint8_t *xb = static_cast<const uint8_t *>(p.x);
+    const int64_t K = p.C, KB = K / 32, KB4 = (K + 127) / 128;
+    const int64_t tiles_c = (KB + TILE_B - 1) / TILE_B;
+    const int64_t tiles_r = ((p.R + 127) / 128) * (128 / TILE_R);
     const int64_t ntiles = tiles_c * tiles_r;
+    const bool a32 = p.aligned32 != 0;
 
-    auto load = [&](int64_t t, uint4(&buf)[RPW]) {
+    auto load = [&](int64_t t, uint32_t(&buf)[RPW][LW]) {
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t c = tc * TILE_C + lane * N;
+        const int64_t b = tc * TILE_B + lane;
         const int64_t r0 = tr * TILE_R + warp * RPW;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
             const int64_t r = r0 + i;
-            buf[i] = (c < p.C && r < p.R && NVFP4_IN_RANGE(r * p.ld + c, N, x_extent(p.R, p.C, p.ld))) ? ldg_stream(x + r * p.ld + c)
-                                                                                        : make_uint4(0u, 0u, 0u, 0u);
+            if (b < KB && r < p.R && NVFP4_IN_RANGE(r * p.ld + b * 32, 32, x_extent(p.R, p.C, p.ld))) {
+                load_block<LW>(xb + (r * p.ld + b * 32) * (int64_t)sizeof(T), a32, buf[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < LW; ++j) buf[i][j] = 0u;
+            }
         }
     };
 
     int64_t t = ntiles - 1 - (int64_t)blockIdx.x;
-    uint4 cur[RPW], nxt[RPW];
+    uint32_t cur[RPW][LW], nxt[RPW][LW];
     if (t >= 0) load(t, cur);
     for (; t >= 0; t -= gridDim.x) {
         const int64_t tn = t - gridDim.x;
         if (tn >= 0) load(tn, nxt);
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t c = tc * TILE_C + lane * N;
-        const bool col_ok = c < p.C;
-        const int half = (int)(tr & 1);
+        const int64_t b = tc * TILE_B + lane, atom = b >> 2;
+        const bool col_ok = b < KB;
 #pragma unroll
         for (int i = 0; i < RPW; ++i) {
-            const int rl = warp * RPW + i;
-            const int64_t r = tr * TILE_R + rl;
-            float v[N];
-            Vec<T>::unpack(cur[i], v);
+            const int64_t r = tr * TILE_R + warp * RPW + i;
+            float v[32];
+            float(&v0)[16] = *reinterpret_cast<float(*)[16]>(v);
+            float(&v1)[16] = *reinterpret_cast<float(*)[16]>(v + 16);
+            unpack16<T>(cur[i], v0);
+            unpack16<T>(cur[i] + LW / 2, v1);
             float m = 0.0f;
 #pragma unroll
-            for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
-#pragma unroll
-            for (int o = 1; o < LPB; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
             const uint32_t code = mx_code(m);
             const float inv = __uint_as_float((254u - code) << 23);  // 2^-X
-            float q[N];
+            float q[32];
 #pragma unroll
-            for (int j = 0; j < N; ++j) q[j] = __fmul_rn(v[j], inv);
-            if (col_ok && r < p.R && NVFP4_IN_RANGE(r * (K / 2) + c / 2, N / 2, p.R * (K / 2))) {
-                uint8_t *dst = p.codes + r * (K / 2) + c / 2;
-                if (N == 8) *reinterpret_cast<uint32_t *>(dst) = e2m1x8(q);
-                else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)e2m1x4(q[0], q[1], q[2], q[3]);
-            }
-            if ((lane % LPB) == 0) {
-                const int ra = half * TILE_R + rl, bl = lane / LPB;  // 32-block within the tile
-                s_sc[(bl >> 2) * 512 + (ra & 31) * 16 + ((ra >> 5) & 3) * 4 + (bl & 3)] = (uint8_t)code;
-            }
+            for (int j = 0; j < 32; ++j) q[j] = __fmul_rn(v[j], inv);
+            if (col_ok && r < p.R && NVFP4_IN_RANGE(r * (K / 2) + b * 16, 16, p.R * (K / 2)))
+                *reinterpret_cast<uint4 *>(p.codes + r * (K / 2) + b * 16) =
+                    make_uint4(e2m1x8(q), e2m1x8(q + 8), e2m1x8(q + 16), e2m1x8(q + 24));
+            uint32_t word = code << (8 * (lane & 3));
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+            if ((lane & 3) == 0 && atom < KB4 &&
+                NVFP4_IN_RANGE(((r >> 7) * KB4 + atom) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4, 4,
+                               mx_scales_extent(p.R, p.C)))
+                *reinterpret_cast<uint32_t *>(p.scales + ((r >> 7) * KB4 + atom) * 512 + (r & 31) * 16 +
+                                              ((r >> 5) & 3) * 4) = word;
         }
-        __syncthreads();
-        const int64_t atom0 = tc * ATOMS;
-        for (int i = threadIdx.x; i < ATOMS * 32; i += kThreads) {
-            const int atom = i >> 5;
-            if (atom0 + atom < KB4 &&
-                NVFP4_IN_RANGE(((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half, 8,
-                               mx_scales_extent(p.R, p.C))) {
-                const int off = atom * 512 + (i & 31) * 16 + 8 * half;
-                uint8_t *dst = p.scales + ((tr >> 1) * KB4 + atom0 + atom) * 512 + (i & 31) * 16 + 8 * half;
-                *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(s_sc + off);
-            }
-        }
-        __syncthreads();
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) cur[i] = nxt[i];
+        for (int i = 0; i < RPW; ++i)
+#pragma unroll
+            for (int j = 0; j < LW; ++j) cur[i][j] = nxt[i][j];
     }
 }
 
@@ -1234,7 +1231,9 @@ cudaError_t launch_quantize_dual(const DualQuantizeArgs &a, cudaStream_t s, int 
 cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, int64_t ld, bool colwise,
                                uint8_t *codes, uint8_t *scales, cudaStream_t s, int *launches) {
     if (R == 0 || C == 0) return cudaSuccess;
-    const MxParams p{x, R, C, ld, codes, scales};
+    MxParams p{x, R, C, ld, codes, scales, 0};
+    const size_t es = bf16 ? 2 : 4;
+    p.aligned32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && ((ld * (int64_t)es) % 32 == 0);
     if (colwise) {
         const int cpt = bf16 ? 4 : 2;
         const int64_t cols_pad = ((C + 127) / 128) * 128, rows_pad = ((R + 127) / 128) * 128;
@@ -1244,8 +1243,8 @@ cudaError_t launch_quantize_mx(const void *x, bool bf16, int64_t R, int64_t C, i
         ++*launches;
         return cudaGetLastError();
     }
-    const int N = bf16 ? Vec<uint16_t>::N : Vec<float>::N;
-    const int64_t tiles = ((C + 32 * N - 1) / (32 * N)) * 2 * ((R + 127) / 128);
+    const int64_t tile_r = bf16 ? 16 : 8;  // rows per tile of quantize_rowwise_mx_kernel
+    const int64_t tiles = ((C / 32 + 31) / 32) * ((R + 127) / 128) * (128 / tile_r);
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, 2 * (int64_t)num_sms());
     if (bf16) quantize_rowwise_mx_kernel<uint16_t><<<grid, kThreads, 0, s>>>(p);
     else quantize_rowwise_mx_kernel<float><<<grid, kThreads, 0, s>>>(p);

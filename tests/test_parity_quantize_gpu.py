@@ -70,6 +70,18 @@ def test_amax_supplied(colwise, cuda_lib):
         check_quantize(x, colwise=colwise, sr=True, amax_in=amax)
 
 
+@pytest.mark.parametrize("mode", [m for m in MODES if m[1]], ids=lambda m: "cw%d-sr%d-rht%d" % m)
+def test_amax_supplied_overflow(mode, cuda_lib):
+    """A supplied amax far below the data's: every block scale saturates at 448, the element
+    scale 1/(448 s_t) stays finite (~1e10) and v / scale overflows to +-inf for most elements,
+    which must encode as +-6 like any |v / scale| >= 6 (the saturation rule of the E2M1 encoding)."""
+    colwise, sr, rht = mode
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((64, 96)) * 1e36).astype(np.float32)
+    for v in (x, W.bf16_bits(x)):
+        check_quantize(v, colwise, sr, rht, seed=5, amax_in=6e-10)
+
+
 def test_e2m1_conversion_sweep(cuda_lib):
     """Every element is rounded at exactly its own value: blocks [6, v1..v15] with a
     supplied amax of 2688 give s_t = 1 and block scale 1, so r = v.  The v sweep covers
