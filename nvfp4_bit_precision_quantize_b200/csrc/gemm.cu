@@ -15,22 +15,25 @@
 // 128 x 256 FP32 accumulator in its own TMEM.  Warp roles, per CTA:
 //   warp 0 (one lane)  producer: TMA loads of this CTA's A and B code tiles
 //                      (128-byte swizzle) and scale atoms (A: its 128 rows;
-//                      B: all 256 rows) into a 5-stage ring; completion bytes
-//                      of both CTAs are counted on the leader's barriers, the
-//                      scale atoms on a barrier of their own;
+//                      B: all 256 rows) into a 5-stage ring; the code bytes of
+//                      both CTAs are counted on the leader's barriers, each
+//                      CTA's scale atoms on a barrier of its own;
 //   warp 1             allocates TMEM (pair-wide); on the leader one lane issues
 //                      the MMAs, four per 256-k stage, reading the stage's
 //                      scales from its TMEM slot; tcgen05.commit multicast to
 //                      both CTAs frees the stage;
-//   warps 11-12        scale copiers (leader), alternate stages: once a stage's
-//                      scale atoms have landed, copy them into the stage's TMEM
-//                      slot (tcgen05.cp, cta_group::2) and commit to the
-//                      stage's scale barrier.  Issued from their own warps,
-//                      the copies (twelve per stage) overlap the MMAs of
-//                      earlier stages instead of queueing in front of them:
-//                      moving them out of the MMA warp took the 8192 x 20480
-//                      x 5120 GEMM from 0.53 to 0.37 ms;
-//   warp 10            waiter (leader): polls the stage's code and scale-copy
+//   warps 11-14        scale writers (both CTAs), one per TMEM lane quarter:
+//                      once a stage's scale atoms have landed, each lane loads
+//                      its row of every atom from shared memory and writes it
+//                      into the stage's TMEM slot with tcgen05.st, in the
+//                      layout a tcgen05.cp 32x128b.warpx4 copy of the atom
+//                      gives; then the warp arrives on the leader's scale
+//                      barrier.  Twelve tcgen05.cp copies per stage from one
+//                      warp took ~930 cycles and finished after the code tiles
+//                      had landed on most stages; the stores take a fraction
+//                      of that and leave the tensor pipe to the MMAs (8192 x
+//                      20480 x 5120: 0.356 -> 0.343 ms, interleaved runs);
+//   warp 10            waiter (leader): polls the stage's code and scale
 //                      barriers and the accumulator-free barrier, and relays
 //                      each event to the
 //                      MMA warp through a hardware named barrier, so that the
@@ -42,15 +45,11 @@
 //                      shared-memory chunk and a TMA store (32 rows x 128
 //                      bytes per chunk; per-row stores from registers cost
 //                      several microseconds per tile here).
-// Scale copies through four extra warps (tcgen05.st from shared memory into
-// per-stage TMEM slots, keeping the MMA warp's pipe free of copies) were
-// measured slower: the extra hop on every stage's refill path cost more than
-// the ~24 tensor-pipe cycles per copy it saves, with five stages in flight.
 // TMEM: accumulator columns [0, 256), then one 48-column scale slot per stage.
 // Tiles are visited in groups of 8 tile columns so that the pairs running at
 // the same time share A and B panels in L2.  Every mbarrier wait is bounded
 // (about 2 s of %globaltimer); on expiry the CTA records
-// NVFP4_ERR_DEVICE_TIMEOUT in the status word, drains its copies and MMAs,
+// NVFP4_ERR_DEVICE_TIMEOUT in the status word, drains its loads and MMAs,
 // frees TMEM and returns.  No TMA load uses cluster multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -80,8 +79,8 @@ constexpr int BAR_OFF = STAGING_OFF + EPI_WARPS * CHUNK_BYTES;
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-constexpr int SF_WARPS = 2;                     // scale copiers, taking alternate k-stages
-constexpr int THREADS = 32 * (11 + SF_WARPS);   // producer, MMA, 8 epilogue warps, waiter, copiers
+constexpr int SF_WARPS = 4;                     // scale writers, one per TMEM lane quarter (both CTAs)
+constexpr int THREADS = 32 * (11 + SF_WARPS);   // producer, MMA, 8 epilogue warps, waiter, scale writers
 constexpr int MMA_WARP = 1, EPI_WARP0 = 2, WAITER_WARP = 10, SF_WARP0 = 11;
 // Hardware named barriers (64 threads: the waiter warp and the MMA warp).
 constexpr uint32_t NB_ACC = 1;     // accumulator free for the next tile
@@ -218,7 +217,9 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 // issue sequence) and issues each tensor-core instruction from the lanes whose
 // `issue` is non-zero -- one lane -- through a PTX predicate.
 // Scale atom (32 rows x 16 bytes in smem) -> 32 TMEM lanes x 4 columns, copied to
-// all four lane quarters, in both CTAs of the pair (each from its own smem).
+// all four lane quarters, in both CTAs of the pair (each from its own smem).  The
+// tensor-pipe probe below loads its scales this way; the GEMM writes the same
+// layout with tcgen05.st.
 __device__ __forceinline__ void tc_cp_scales_if(uint32_t issue, uint32_t taddr, uint64_t sdesc) {
     asm volatile(
         "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t"
@@ -300,6 +301,25 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[3
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 16 / 32 consecutive TMEM columns of this warp's lane quarter from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *w) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+        "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *w) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+        "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15]), "r"(w[16]), "r"(w[17]), "r"(w[18]),
+        "r"(w[19]), "r"(w[20]), "r"(w[21]), "r"(w[22]), "r"(w[23]), "r"(w[24]), "r"(w[25]), "r"(w[26]), "r"(w[27]),
+        "r"(w[28]), "r"(w[29]), "r"(w[30]), "r"(w[31])
+        : "memory");
+}
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart (SBO); LBO unused; version 1 (sm_100).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
@@ -419,10 +439,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t bar_acce = smem_u32(bars + 2 * STAGES + 1);   // leader: accumulator read (16 epilogue warps)
     const uint32_t bar_drain = smem_u32(bars + 2 * STAGES + 2);  // leader: every MMA done
     const uint32_t bar_epi = smem_u32(bars + 2 * STAGES + 3);    // [8] each CTA: an epilogue warp's aux chunk
-    const uint32_t bar_sf = smem_u32(bars + 2 * STAGES + 3 + EPI_WARPS);          // [S] leader: stage's scales in TMEM
-    const uint32_t bar_sf_drain = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS);    // [2] leader: a copier's copies done
-    const uint32_t bar_sfull = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS + SF_WARPS);  // [S] leader: scale bytes
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 3 + EPI_WARPS + SF_WARPS);
+    const uint32_t bar_sf = smem_u32(bars + 2 * STAGES + 3 + EPI_WARPS);       // [S] leader: stage's scales in TMEM
+    const uint32_t bar_sfull = smem_u32(bars + 3 * STAGES + 3 + EPI_WARPS);    // [S] each CTA: its scale bytes
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 3 + EPI_WARPS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *stop_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);  // waiter -> MMA warp, per tile
     float *red = reinterpret_cast<float *>(tmem_slot + 4);                      // fused amax: 2 x 8 warps
@@ -436,10 +455,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
-            mbar_init(bar_sf + 8 * s, 1);
+            mbar_init(bar_sf + 8 * s, 2 * SF_WARPS);  // the scale writers of both CTAs
             mbar_init(bar_sfull + 8 * s, 1);
         }
-        for (int c = 0; c < SF_WARPS; ++c) mbar_init(bar_sf_drain + 8 * c, 1);
         mbar_init(bar_accf, 1);
         mbar_init(bar_acce, 2 * EPI_WARPS);
         mbar_init(bar_drain, 1);
@@ -470,8 +488,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
             uint32_t s = 0, ph = 0;
             bool ok = true;
-            // Bytes per CTA per stage: the scale atoms complete on their own barrier, so
-            // that the copiers can move them into TMEM while the codes still land.
+            // Bytes per CTA per stage: the scale atoms complete on a barrier of this CTA,
+            // so that its scale writers can move them into TMEM while the codes still land.
             constexpr uint32_t CODES_TX = A_BYTES + B_BYTES, SCALES_TX = 3 * APS * 512;
             for (int t = cid; t < p.num_tiles && ok; t += ncl) {
                 int mt, nt;
@@ -485,18 +503,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     const uint32_t st = smem_base + s * STAGE_BYTES;
                     const uint32_t full_leader = mapa(bar_full + 8 * s, 0);
-                    const uint32_t sfull_leader = mapa(bar_sfull + 8 * s, 0);
                     // Out-of-range rows, columns and atoms are zero-filled and still
                     // counted, so every stage brings exactly CODES_TX + SCALES_TX bytes
                     // per CTA.
-                    if (rank == 0) {
-                        mbar_expect_tx(bar_sfull + 8 * s, 2 * SCALES_TX);
-                        mbar_expect_tx(bar_full + 8 * s, 2 * CODES_TX);
-                    }
-                    tma_load_pair(st + SF_OFF, &map_sfa, sfull_leader, 0, ya + kt * APS, policy);
-                    tma_load_pair(st + SF_OFF + SFA_BYTES, &map_sfb, sfull_leader, 0, yb + kt * APS, policy);
-                    tma_load_pair(st + SF_OFF + SFA_BYTES + 2048, &map_sfb, sfull_leader, 0, yb + p.kbs + kt * APS,
-                                  policy);
+                    mbar_expect_tx(bar_sfull + 8 * s, SCALES_TX);
+                    if (rank == 0) mbar_expect_tx(bar_full + 8 * s, 2 * CODES_TX);
+                    tma_load_own(st + SF_OFF, &map_sfa, bar_sfull + 8 * s, 0, ya + kt * APS, policy);
+                    tma_load_own(st + SF_OFF + SFA_BYTES, &map_sfb, bar_sfull + 8 * s, 0, yb + kt * APS, policy);
+                    tma_load_own(st + SF_OFF + SFA_BYTES + 2048, &map_sfb, bar_sfull + 8 * s, 0,
+                                 yb + p.kbs + kt * APS, policy);
                     tma_load_pair(st, &map_a, full_leader, kt * (BK / 2), m0, policy);
                     tma_load_pair(st + A_BYTES, &map_b, full_leader, kt * (BK / 2), n0 + 128 * (int)rank, policy);
                     if (++s == STAGES) {
@@ -505,7 +520,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                 }
             }
-            // This CTA's loads complete on the leader's barriers; the leader drains them.
+            // This CTA's code tiles complete on the leader's barriers, and the leader drains
+            // them; its scale atoms on its own, which its scale writers drain.
         }
     } else if (warp == MMA_WARP) {
         if (rank == 0) {
@@ -523,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 uint32_t acc = 0;  // the first MMA of a tile overwrites the accumulator
                 for (int kt = 0; kt < num_kt; ++kt) {
                     // Stage s has landed and its scales are in TMEM slot s (the waiter saw
-                    // the scale copier's barrier complete).
+                    // the scale writers' barrier complete).
                     named_sync(NB_STAGE0 + s);
                     tc_fence_after();
                     const uint32_t sa = smem_base + s * STAGE_BYTES;
@@ -583,8 +599,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (rank == 0) {
             // ---------------- waiter (leader only) ----------------
             // Waits on the accumulator-free barrier and, per stage, on its code bytes
-            // and on its scale barrier (a copier signals it once the stage's scale
-            // atoms reached TMEM) in the order the MMA warp consumes them, and relays
+            // and on its scale barrier (the scale writers of both CTAs arrive once the
+            // stage's scale atoms are in TMEM) in the order the MMA warp consumes them, and relays
             // each through a named barrier.  After
             // a timeout inside a tile it keeps relaying without waiting until the
             // tile ends, then both warps stop.
@@ -603,7 +619,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (stop) break;
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (ok) ok = mbar_wait_warp(bar_full + 8 * s, ph, abort_flag);
-                    if (ok) ok = mbar_wait_warp(bar_sf + 8 * s, ph, abort_flag);
+                    if (ok) ok = mbar_wait_warp<true>(bar_sf + 8 * s, ph, abort_flag);  // writers of both CTAs
                     named_sync(NB_STAGE0 + s);
                     if (++s == STAGES) {
                         s = 0;
@@ -613,53 +629,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
         }
     } else if (warp >= SF_WARP0 && warp < SF_WARP0 + SF_WARPS) {
-        if (rank == 0) {
-            // ---------------- scale copiers (leader's warps 11-12, lane 0 issues) ----------------
-            // Copier c takes the k-stages i with i % 2 == c: once stage s's scale
-            // atoms have landed (bar_sfull, usually before the code tiles), they go
-            // into TMEM slot s (tcgen05.cp, both CTAs), then a commit arrives on
-            // bar_sf[s] when the copies are done.  A copy occupies
-            // its issuing warp for ~70 cycles, so one warp alone needs ~850 cycles per
-            // stage, against 512 for the stage's four MMAs; two warps keep ahead of
-            // the MMA warp.  Slot s is free again once stage s's scales have landed
-            // anew: the producer refills the stage only after the MMAs that read the
-            // slot have completed.
-            const int mine = warp - SF_WARP0;
-            const uint32_t issue = lane == 0 ? 1u : 0u;
-            uint32_t s = 0, ph = 0;
-            bool ok = true;
-            int it = 0;
-            for (int t = cid; t < p.num_tiles && ok; t += ncl) {
-                for (int kt = 0; kt < num_kt; ++kt, ++it) {
-                    if (it % SF_WARPS == mine) {
-                        if (!mbar_wait_warp(bar_sfull + 8 * s, ph, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t sa = smem_base + s * STAGE_BYTES;
-                        const uint64_t dsa = sdesc_scales(sa + SF_OFF);
-                        const uint64_t dsb = sdesc_scales(sa + SF_OFF + SFA_BYTES);
-                        const uint32_t sf = tmem + TMEM_SF + SF_SLOT_COLS * s;
-                        // Descriptor addresses in 16-byte units: +32 per 512-byte atom,
-                        // +128 for B's second 128-row tile.
-                        const int steps = kt < p.kfull ? 4 : p.ktail;
-                        const int atoms = MX ? (steps + 1) / 2 : steps;
-                        for (int j = 0; j < atoms; ++j) {
-                            tc_cp_scales_if(issue, sf + 4 * j, dsa + 32 * j);
-                            tc_cp_scales_if(issue, sf + 16 + 8 * j, dsb + 32 * j);
-                            tc_cp_scales_if(issue, sf + 20 + 8 * j, dsb + 128 + 32 * j);
-                        }
-                        tc_commit_self_if(issue, bar_sf + 8 * s);
-                    }
-                    if (++s == STAGES) {
-                        s = 0;
-                        ph ^= 1;
-                    }
+        // ---------------- scale writers (both CTAs, warps 11-14) ----------------
+        // Warp w writes TMEM lane quarter w % 4 of its CTA.  Once stage s's scale atoms
+        // have landed in this CTA (bar_sfull, usually well before the code tiles), lane
+        // r loads row r of every atom (16 bytes: the 4-byte words of rows r, r + 32,
+        // r + 64, r + 96) and stores it into 4 columns of lane 32 q + r of the stage's
+        // TMEM slot -- the layout a 32x128b.warpx4 copy of the atom produces, which the
+        // MMA reads -- then arrives on the leader's bar_sf[s] (8 arrivals: four warps in
+        // each CTA).  A whole slot is written every stage (MXFP4 stages, and the short
+        // last stage, leave some of it unread).  The slot is free: the producer reloads
+        // stage s only after the MMAs that read the slot have completed.  These stores
+        // do not queue on the tensor pipe as tcgen05.cp copies do (~930 cycles per stage
+        // from one warp, on the refill path of every stage).
+        const uint32_t q = warp & 3;
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        int it = 0;
+        for (int t = cid; t < p.num_tiles && ok; t += ncl) {
+            for (int kt = 0; kt < num_kt; ++kt, ++it) {
+                if (!mbar_wait_warp(bar_sfull + 8 * s, ph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = smem_base + s * STAGE_BYTES + SF_OFF + (uint32_t)lane * 16u;
+                uint32_t w[48];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {  // SFA atom j -> columns 4 j .. 4 j + 3
+                    const uint4 v = ld_shared_v4(sa + 512u * j);
+                    w[4 * j] = v.x, w[4 * j + 1] = v.y, w[4 * j + 2] = v.z, w[4 * j + 3] = v.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {  // SFB atom j: rows 0-127 -> 16 + 8 j, rows 128-255 -> 20 + 8 j
+                    const uint4 lo = ld_shared_v4(sa + SFA_BYTES + 512u * j);
+                    const uint4 hi = ld_shared_v4(sa + SFA_BYTES + 2048u + 512u * j);
+                    w[16 + 8 * j] = lo.x, w[17 + 8 * j] = lo.y, w[18 + 8 * j] = lo.z, w[19 + 8 * j] = lo.w;
+                    w[20 + 8 * j] = hi.x, w[21 + 8 * j] = hi.y, w[22 + 8 * j] = hi.z, w[23 + 8 * j] = hi.w;
+                }
+                const uint32_t ta = tmem + ((q * 32u) << 16) + TMEM_SF + SF_SLOT_COLS * s;
+                tmem_st16(ta, w);
+                tmem_st32(ta + 16, w + 16);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa(bar_sf + 8 * s, 0));
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1;
                 }
             }
-            tc_commit_self_if(issue, bar_sf_drain + 8 * mine);
-            mbar_wait_warp(bar_sf_drain + 8 * mine, 0, abort_flag, false);  // every copy done before TMEM is freed
+        }
+        if (!ok && warp == SF_WARP0) {
+            // Stages this CTA's producer may still be filling: wait (briefly) for their atoms.
+            for (int k = it; k < it + STAGES; ++k)
+                mbar_wait_warp(bar_sfull + 8 * (k % STAGES), (k / STAGES) & 1, abort_flag, false, DRAIN_LIMIT_NS);
         }
     } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // ---------------- epilogue (both CTAs) ----------------
