@@ -24,7 +24,7 @@ def run_gemm(a, b, out_dtype=torch.float32):
 
 
 SHAPES = [(256, 256, 256), (128, 256, 64), (1, 8, 64), (200, 392, 320), (384, 640, 1024), (520, 264, 2112),
-          (1000, 1000, 1024)]
+          (1000, 1000, 1024), (300, 520, 640), (264, 392, 704)]  # K % 256 = 0, 64, 128, 192: every stage length
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "%dx%dx%d" % s)

@@ -49,7 +49,8 @@ def test_mx_gemm_256_cube(cuda_lib):
     assert_gemm_close(run(a, b).cpu().numpy(), ref, ab, "256^3")
 
 
-SHAPES = [(1, 8, 64), (128, 256, 64), (200, 392, 320), (384, 640, 1024), (520, 264, 2112), (1000, 1000, 1088)]
+SHAPES = [(1, 8, 64), (128, 256, 64), (200, 392, 320), (384, 640, 1024), (520, 264, 2112), (1000, 1000, 1088),
+          (300, 520, 640), (264, 392, 704)]  # K % 256 = 0, 64, 128, 192: every stage length
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "%dx%dx%d" % s)
